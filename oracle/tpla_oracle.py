@@ -1,0 +1,386 @@
+"""CPU float64 oracle for MLA latent-KV decode attention and its TPLA variant.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+execute this module: only the tests, the ``smoke()`` entry point and the
+CPU-baseline leg of ``bench.py`` use it.  It shares no code with the CUDA path
+(no kernels, headers, helpers or constants); both sides only see the same
+seeded input arrays.
+
+Everything here is the plain definition, written out in float64 NumPy with no
+blocking, fusion or reordering beyond what the definitions state.  Inputs are
+the bf16 values of the GPU inputs widened exactly to float64; ``scale`` is the
+float32 value the caller passes, widened.
+
+Sources (web pages on TPLA / MLA latent-cache sharding):
+
+* [ISSUE]  "[Feature Request] Bandwidth-optimal tensor-parallel sharding of MLA
+  (latent-cache sharding / TPLA)", sections "Background / problem",
+  "Directions under investigation", "Methodology (first step)",
+  "Tests / validation".
+* [ABSTRACT] "TPLA: Tensor Parallel Latent Attention for Efficient
+  Disaggregated Prefill & Decode Inference", abstract.
+* [VERDICT] pith.science review of arXiv 2508.15881: skeptic critique
+  (load-bearing attack on Eq. 6), referee report (significance; major comments
+  on Eq. 22/25), pith extraction (key machinery), desk-editor letter.
+
+Readings taken where the pages are silent (each is listed in the design doc):
+
+1. Eq. 6 is not printed; the reviewers state it is an *unscaled* local
+   softmax.  Shard g therefore uses the same ``scale`` as exact MLA and no
+   mu/nu factors.
+2. Shard g owns the contiguous latent columns [g*d, (g+1)*d), d = 512/G.
+3. Rope columns are replicated to every shard ("320 = 256 + 64 at TP=2");
+   the ``split`` rope mode gives shard g the contiguous rope slice
+   [512 + g*64/G, 512 + (g+1)*64/G).
+4. Values are latent columns only (the rope part is key-only in MLA); the
+   output lives in latent space.
+5. Shard outputs are concatenated in shard order; the all-reduce becomes a
+   sum over shards inside the V up-projection.
+6. lse is the natural log of sum(exp(scale * logits)); an empty request has
+   output 0 and lse = -inf.
+7. The Hadamard transform is the orthonormal Sylvester (natural-order) matrix
+   applied to the first ``dim`` columns of a row.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+LATENT = 512  # kv_lora_rank: the latent part of a cache row
+ROPE = 64     # decoupled rope key part of a cache row
+WIDTH = LATENT + ROPE  # 576 values per token ([ISSUE] "Background / problem")
+BLOCK = 64    # tokens per cache page
+
+
+# ---------------------------------------------------------------------------
+# Column bookkeeping for the TPLA shards
+# ---------------------------------------------------------------------------
+
+def shard_columns(G: int, g: int, rope_mode: str = "replicate"):
+    """Return (latent_cols, rope_cols) of shard ``g`` out of ``G``.
+
+    [ABSTRACT]: TPLA partitions the latent representation and each head's
+    input dimension across devices.  [VERDICT referee_report.significance]:
+    the per-device cache is 256 + 64 = 320 dims at TP=2, so the rope part is
+    replicated to every shard.  ``split`` (rope also cut into G slices) is
+    the alternative reading; contiguous slices in shard order (readings 2, 3).
+    """
+    if LATENT % G:
+        raise ValueError("G must divide 512")
+    d = LATENT // G
+    lat = np.arange(g * d, (g + 1) * d)
+    if rope_mode == "replicate":
+        rope = np.arange(LATENT, WIDTH)
+    elif rope_mode == "split":
+        if ROPE % G:
+            raise ValueError("split rope needs G | 64")
+        r = ROPE // G
+        rope = np.arange(LATENT + g * r, LATENT + (g + 1) * r)
+    else:
+        raise ValueError(rope_mode)
+    return lat, rope
+
+
+# ---------------------------------------------------------------------------
+# Cache addressing (pure indexing, no arithmetic of the method)
+# ---------------------------------------------------------------------------
+
+def gather_request_rows(cache, seq_lens, page_table=None):
+    """Return a list with the [L_b, 576] float64 cache rows of each request.
+
+    Paged: token t of request b lives in block ``page_table[b][t // 64]`` at
+    row ``t % 64`` of a [num_blocks, 64, 576] cache.  Contiguous: a
+    [B, Lmax, 576] cache, request b's first L_b rows.
+    """
+    cache = np.asarray(cache)
+    rows = []
+    for b, L in enumerate(np.asarray(seq_lens).tolist()):
+        if page_table is None:
+            rows.append(np.asarray(cache[b, :L], dtype=np.float64))
+        else:
+            t = np.arange(L)
+            blk = np.asarray(page_table)[b][t // BLOCK]
+            rows.append(np.asarray(cache[blk, t % BLOCK], dtype=np.float64))
+    return rows
+
+
+# ---------------------------------------------------------------------------
+# The attention primitive: softmax attention of a few query rows
+# ---------------------------------------------------------------------------
+
+def attention_ref(qh, keys, values, scale):
+    """Softmax attention for one request and one key/value column set.
+
+    qh [H, K], keys [L, K], values [L, V].  s = scale * qh keys^T,
+    out = softmax(s) values, lse = log sum exp(s) (natural log).
+    An empty key set gives out = 0, lse = -inf (reading 6).
+    """
+    qh = np.asarray(qh, dtype=np.float64)
+    H = qh.shape[0]
+    V = values.shape[1]
+    if keys.shape[0] == 0:
+        return np.zeros((H, V)), np.full((H,), -np.inf)
+    s = float(scale) * (qh @ np.asarray(keys, dtype=np.float64).T)  # [H, L]
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    z = p.sum(axis=1, keepdims=True)
+    out = (p @ np.asarray(values, dtype=np.float64)) / z
+    lse = (m + np.log(z))[:, 0]
+    return out, lse
+
+
+def attention_bruteforce(qh, keys, values, scale):
+    """Scalar-loop restatement of ``attention_ref`` for tiny inputs.
+
+    Pure Python floats and ``math.exp``; used only to pin the NumPy version.
+    """
+    H = len(qh)
+    L = len(keys)
+    V = len(values[0]) if L else 0
+    out = [[0.0] * V for _ in range(H)]
+    lse = [-math.inf] * H
+    for h in range(H):
+        if L == 0:
+            continue
+        s = []
+        for t in range(L):
+            acc = 0.0
+            for j in range(len(qh[h])):
+                acc += float(qh[h][j]) * float(keys[t][j])
+            s.append(float(scale) * acc)
+        m = max(s)
+        w = [math.exp(x - m) for x in s]
+        z = sum(w)
+        for v in range(V):
+            out[h][v] = sum(w[t] * float(values[t][v]) for t in range(L)) / z
+        lse[h] = m + math.log(z)
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Exact MLA decode (absorbed form) and TPLA
+# ---------------------------------------------------------------------------
+
+def mla_decode_ref(q, rows, scale):
+    """Exact absorbed MLA decode: one new token per request.
+
+    Every head attends over all 576 cached values per token (512 latent +
+    64 rope; [ISSUE] "Background / problem") with one softmax; values are
+    the 512 latent columns, so the output stays in latent space.
+    q [B, H, 576]; rows: per-request [L_b, 576].  Returns out [B, H, 512],
+    lse [B, H].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, H, _ = q.shape
+    out = np.zeros((B, H, LATENT))
+    lse = np.zeros((B, H))
+    for b in range(B):
+        c = rows[b]
+        out[b], lse[b] = attention_ref(q[b], c, c[:, :LATENT], scale)
+    return out, lse
+
+
+def tpla_decode_ref(q, rows, G, rope_mode, scale, shard=None):
+    """TPLA decode: G latent shards, an independent softmax per shard.
+
+    [ISSUE] "Directions under investigation": each rank runs local attention
+    over its latent slice.  [VERDICT pith_extraction.key_machinery]: device i
+    computes softmax(Q_i (cKV_i U)^T) with all query heads replicated;
+    [VERDICT skeptic_critique]: Eq. 6 is an unscaled local softmax.
+    Shard g's logits use its latent columns plus its rope columns; its
+    values are its latent columns only.  Outputs are concatenated in shard
+    order (reading 5).
+
+    Returns out [B, H, 512] and lse [B, H, G].  With ``shard = s`` (one-shard
+    mode: the work of one TP rank) returns out [B, H, d] and lse [B, H, 1].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, H, _ = q.shape
+    d = LATENT // G
+    shards = range(G) if shard is None else [shard]
+    width = LATENT if shard is None else d
+    out = np.zeros((B, H, width))
+    lse = np.zeros((B, H, len(shards)))
+    for b in range(B):
+        c = rows[b]
+        for k, g in enumerate(shards):
+            lat, rope = shard_columns(G, g, rope_mode)
+            cols = np.concatenate([lat, rope])
+            o, l = attention_ref(q[b][:, cols], c[:, cols], c[:, lat], scale)
+            if shard is None:
+                out[b][:, lat] = o
+            else:
+                out[b] = o
+            lse[b, :, k] = l
+    return out, lse
+
+
+def gla_decode_ref(q, rows, G, rope_mode, scale):
+    """TPLA written as Grouped Latent Attention with G*H heads.
+
+    [VERDICT desk_editor.letter / pith_summary]: TPLA is a special case of
+    GLA with replicated heads.  Head (g, h) of the GLA model sees latent group
+    g only.  This restatement builds the grouped keys explicitly, evaluates
+    all G*H heads in one batched contraction and normalises with SciPy's
+    ``logsumexp``, so it shares no softmax code with ``tpla_decode_ref``.
+    Returns out [B, H, 512], lse [B, H, G].
+    """
+    from scipy.special import logsumexp
+
+    q = np.asarray(q, dtype=np.float64)
+    B, H, _ = q.shape
+    d = LATENT // G
+    groups = [shard_columns(G, g, rope_mode) for g in range(G)]
+    kdim = d + len(groups[0][1])
+    out = np.zeros((B, H, LATENT))
+    lse = np.zeros((B, H, G))
+    for b in range(B):
+        c = rows[b]
+        L = c.shape[0]
+        # grouped query [G*H, kdim] and grouped keys/values [G, L, *]
+        qg = np.stack([q[b][:, np.concatenate(groups[g])] for g in range(G)])
+        kg = np.stack([c[:, np.concatenate(groups[g])] for g in range(G)])
+        vg = np.stack([c[:, groups[g][0]] for g in range(G)])
+        if L == 0:
+            lse[b] = -np.inf
+            continue
+        s = float(scale) * np.einsum("ghk,glk->ghl", qg, kg)  # [G, H, L]
+        ls = logsumexp(s, axis=2)  # [G, H]
+        w = np.exp(s - ls[..., None])
+        o = np.einsum("ghl,glv->ghv", w, vg)  # [G, H, d]
+        for g in range(G):
+            out[b][:, g * d:(g + 1) * d] = o[g]
+            lse[b, :, g] = ls[g]
+    return out, lse
+
+
+def tpla_decode_paged_ref(q, cache, seq_lens, page_table, G, rope_mode,
+                          scale, shard=None):
+    """``tpla_decode_ref`` on a paged ([num_blocks, 64, 576]) or contiguous
+    ([B, Lmax, 576], ``page_table=None``) cache."""
+    rows = gather_request_rows(cache, seq_lens, page_table)
+    return tpla_decode_ref(q, rows, G, rope_mode, scale, shard)
+
+
+# ---------------------------------------------------------------------------
+# Sequence split + log-sum-exp merge
+# ---------------------------------------------------------------------------
+
+def lse_merge_ref(o_parts, lse_parts):
+    """Merge attention results of disjoint key chunks.
+
+    [ISSUE] "Directions under investigation": the exact context/sequence
+    parallel alternative splits the sequence and merges with the
+    flash-attention log-sum-exp rule.  o_parts [S, ..., V] (each chunk's
+    normalised output), lse_parts [S, ...].  lse = log sum_k exp(lse_k),
+    out = sum_k exp(lse_k - lse) o_k.  Chunks with lse = -inf weigh 0; if
+    all are -inf the result is out 0, lse -inf.
+    """
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    M = lse_parts.max(axis=0)
+    finite = np.isfinite(M)
+    Ms = np.where(finite, M, 0.0)
+    w = np.where(np.isfinite(lse_parts), np.exp(lse_parts - Ms), 0.0)
+    z = w.sum(axis=0)
+    lse = np.where(finite, Ms + np.log(np.where(finite, z, 1.0)), -np.inf)
+    zz = np.where(finite, z, 1.0)
+    out = (w[..., None] * o_parts).sum(axis=0) / zz[..., None]
+    out = np.where(finite[..., None], out, 0.0)
+    return out, lse
+
+
+def split_decode_ref(q, rows, G, rope_mode, scale, bounds):
+    """TPLA decode with each request's tokens cut at ``bounds`` (a sorted list
+    of token offsets starting at 0 and ending at L_b or beyond) and merged
+    with ``lse_merge_ref``.  Used to check that the split path is exact."""
+    q = np.asarray(q, dtype=np.float64)
+    B, H, _ = q.shape
+    outs, lses = [], []
+    for k in range(len(bounds) - 1):
+        chunk = [r[bounds[k]:bounds[k + 1]] for r in rows]
+        o, l = tpla_decode_ref(q, chunk, G, rope_mode, scale)
+        d = LATENT // G
+        # per-shard merge: lay each shard's lse next to its columns
+        outs.append(o.reshape(B, H, G, d))
+        lses.append(l)
+    o, l = lse_merge_ref(np.stack(outs), np.stack(lses))
+    return o.reshape(B, H, LATENT), l
+
+
+# ---------------------------------------------------------------------------
+# Orthogonal (Walsh-Hadamard) reparameterisation
+# ---------------------------------------------------------------------------
+
+def hadamard_matrix(n: int):
+    """Orthonormal Sylvester Hadamard matrix, natural order:
+    H[i, j] = (-1)^popcount(i & j) / sqrt(n)  (reading 7).
+
+    [ISSUE] "Directions under investigation" and [ABSTRACT]: an orthogonal
+    transform (Hadamard or PCA) applied to the latent before TP slicing.
+    """
+    if n <= 0 or n & (n - 1):
+        raise ValueError("n must be a power of two")
+    i = np.arange(n)
+    parity = np.zeros((n, n), dtype=np.int64)
+    x = i[:, None] & i[None, :]
+    while np.any(x):
+        parity ^= x & 1
+        x = x >> 1
+    return np.where(parity == 1, -1.0, 1.0) / math.sqrt(n)
+
+
+def hadamard_ref(x, dim):
+    """Apply the orthonormal Hadamard transform to the first ``dim`` columns
+    of every row of ``x`` (rows are the last axis); other columns unchanged."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    Hm = hadamard_matrix(dim)
+    x[..., :dim] = x[..., :dim] @ Hm  # H is symmetric: row-vector form
+    return x
+
+
+# ---------------------------------------------------------------------------
+# V up-projection combine (stands in for the o_proj all-reduce)
+# ---------------------------------------------------------------------------
+
+def vup_ref(out_latent, W_uv):
+    """y[b, h, :] = sum_j out[b, h, j] W_uv[h, j, :].
+
+    [ISSUE] "Directions under investigation": shard outputs are combined by
+    the existing o_proj all-reduce; with shards laid side by side in latent
+    space that sum over shards is the contraction over j (reading 5).
+    out_latent [B, H, 512], W_uv [H, 512, Dv] -> y [B, H, Dv].
+    """
+    return np.einsum("bhj,hjk->bhk", np.asarray(out_latent, np.float64),
+                     np.asarray(W_uv, np.float64))
+
+
+def vup_sharded_ref(out_latent, W_uv, G):
+    """The same combine written as the pages describe the deployment: each
+    shard's partial product out_g W_uv[h, I_g, :], then a sum over shards
+    (the all-reduce)."""
+    out_latent = np.asarray(out_latent, np.float64)
+    W_uv = np.asarray(W_uv, np.float64)
+    d = LATENT // G
+    parts = [np.einsum("bhj,hjk->bhk", out_latent[:, :, g * d:(g + 1) * d],
+                       W_uv[:, g * d:(g + 1) * d, :]) for g in range(G)]
+    return np.sum(parts, axis=0)
+
+
+# ---------------------------------------------------------------------------
+# Diagnostics (informational only; never pass/fail)
+# ---------------------------------------------------------------------------
+
+def per_head_cosine(a, b):
+    """Cosine similarity per (request, head) of two [B, H, V] outputs.
+
+    [VERDICT skeptic_critique.concrete_test] proposes the per-head cosine of
+    the TPLA output against exact MLA as the direct fidelity measurement.
+    """
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    num = (a * b).sum(-1)
+    den = np.linalg.norm(a, axis=-1) * np.linalg.norm(b, axis=-1)
+    return num / np.where(den == 0, 1.0, den)

@@ -1,0 +1,354 @@
+"""Pins for the CPU float64 oracle: each test checks it against something
+other than itself (brute force, closed forms, library routines, invariants
+the pages state).  CPU only."""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import tpla_oracle as O
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SCALE = np.float64(np.float32(1.0 / math.sqrt(192.0)))
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _rows(B, Ls, seed):
+    rng = np.random.default_rng(seed)
+    return [rng.standard_normal((L, O.WIDTH)) for L in Ls]
+
+
+# ---------------------------------------------------------------- page figures
+
+def test_page_figures_widths():
+    fig = json.load(open(os.path.join(HERE, "golden", "page_figures.json")))
+    assert O.WIDTH == fig["values_per_token_mla"]["value"]
+    assert O.LATENT == fig["latent_dims"]["value"]
+    # one TP=2 rank reads its 256 latent columns plus the replicated rope
+    for g in range(2):
+        lat, rope = O.shard_columns(2, g, "replicate")
+        assert len(lat) + len(rope) == fig["values_per_device_tpla_tp2"]["value"]
+
+
+def test_shard_columns_partition():
+    for G in (1, 2, 4, 8):
+        lat_all = np.concatenate([O.shard_columns(G, g)[0] for g in range(G)])
+        assert np.array_equal(lat_all, np.arange(512))
+        for g in range(G):
+            assert np.array_equal(O.shard_columns(G, g, "replicate")[1],
+                                  np.arange(512, 576))
+    for G in (1, 2, 4):
+        rope_all = np.concatenate([O.shard_columns(G, g, "split")[1] for g in range(G)])
+        assert np.array_equal(rope_all, np.arange(512, 576))
+
+
+# ---------------------------------------------------------------- brute force
+
+@pytest.mark.parametrize("H,L,K,V", [(1, 1, 3, 2), (3, 7, 5, 4), (4, 16, 9, 6)])
+def test_attention_matches_bruteforce(H, L, K, V):
+    q = _rand((H, K), 1)
+    keys = _rand((L, K), 2)
+    vals = _rand((L, V), 3)
+    o, l = O.attention_ref(q, keys, vals, 0.7)
+    ob, lb = O.attention_bruteforce(q.tolist(), keys.tolist(), vals.tolist(), 0.7)
+    assert np.allclose(o, np.array(ob), rtol=1e-13, atol=1e-13)
+    assert np.allclose(l, np.array(lb), rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("G,rope_mode", [(1, "replicate"), (2, "replicate"),
+                                         (2, "split"), (4, "split")])
+def test_tpla_matches_bruteforce_hardcoded_columns(G, rope_mode):
+    """Shard column sets written out here from the definition (not through
+    shard_columns), then a scalar-loop softmax per shard."""
+    B, H, L = 1, 2, 5
+    q = _rand((B, H, O.WIDTH), 11)
+    rows = _rows(B, [L], 12)
+    out, lse = O.tpla_decode_ref(q, rows, G, rope_mode, SCALE)
+    d = 512 // G
+    for g in range(G):
+        lat = list(range(g * d, g * d + d))
+        if rope_mode == "replicate":
+            rope = list(range(512, 576))
+        else:
+            r = 64 // G
+            rope = list(range(512 + g * r, 512 + g * r + r))
+        cols = lat + rope
+        qh = [[q[0, h, j] for j in cols] for h in range(H)]
+        keys = [[rows[0][t, j] for j in cols] for t in range(L)]
+        vals = [[rows[0][t, j] for j in lat] for t in range(L)]
+        ob, lb = O.attention_bruteforce(qh, keys, vals, SCALE)
+        assert np.allclose(out[0][:, lat], np.array(ob), rtol=1e-12, atol=1e-12)
+        assert np.allclose(lse[0, :, g], np.array(lb), rtol=1e-12, atol=1e-12)
+
+
+def test_mla_matches_bruteforce():
+    B, H, L = 1, 3, 6
+    q = _rand((B, H, O.WIDTH), 21)
+    rows = _rows(B, [L], 22)
+    out, lse = O.mla_decode_ref(q, rows, SCALE)
+    keys = rows[0].tolist()
+    vals = rows[0][:, :512].tolist()
+    ob, lb = O.attention_bruteforce(q[0].tolist(), keys, vals, SCALE)
+    assert np.allclose(out[0], np.array(ob), rtol=1e-12, atol=1e-12)
+    assert np.allclose(lse[0], np.array(lb), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- invariants
+
+def test_g1_equals_exact_mla():
+    """'G=1 matches head-TP MLA exactly' (issue, Tests / validation)."""
+    B, H = 3, 4
+    q = _rand((B, H, O.WIDTH), 31)
+    rows = _rows(B, [9, 1, 33], 32)
+    o1, l1 = O.tpla_decode_ref(q, rows, 1, "replicate", SCALE)
+    om, lm = O.mla_decode_ref(q, rows, SCALE)
+    # identical up to the summation order BLAS picks for the gathered columns
+    assert np.allclose(o1, om, rtol=1e-13, atol=1e-14)
+    assert np.allclose(l1[..., 0], lm, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("G,rope_mode", [(2, "replicate"), (4, "replicate"),
+                                         (2, "split"), (4, "split"), (8, "replicate")])
+def test_tpla_equals_gla_with_replicated_heads(G, rope_mode):
+    """TPLA == GLA with G*H heads (review, desk-editor letter)."""
+    B, H = 2, 3
+    q = _rand((B, H, O.WIDTH), 41)
+    rows = _rows(B, [17, 40], 42)
+    ot, lt = O.tpla_decode_ref(q, rows, G, rope_mode, SCALE)
+    og, lg = O.gla_decode_ref(q, rows, G, rope_mode, SCALE)
+    assert np.allclose(ot, og, rtol=1e-12, atol=1e-13)
+    assert np.allclose(lt, lg, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("G,rope_mode", [(1, "replicate"), (2, "replicate"), (4, "split")])
+def test_constant_cache_returns_row(G, rope_mode):
+    """All cached rows equal r: softmax weights sum to one, so every shard
+    returns r's latent slice; lse = scale * q.r + ln L."""
+    B, H, L = 2, 5, 13
+    q = _rand((B, H, O.WIDTH), 51)
+    r = _rand((O.WIDTH,), 52)
+    rows = [np.tile(r, (L, 1)) for _ in range(B)]
+    out, lse = O.tpla_decode_ref(q, rows, G, rope_mode, SCALE)
+    for b in range(B):
+        assert np.allclose(out[b], np.tile(r[:512], (H, 1)), rtol=1e-12, atol=1e-12)
+        for g in range(G):
+            lat, rope = O.shard_columns(G, g, rope_mode)
+            cols = np.concatenate([lat, rope])
+            expect = SCALE * (q[b][:, cols] @ r[cols]) + math.log(L)
+            assert np.allclose(lse[b, :, g], expect, rtol=1e-12, atol=1e-12)
+
+
+def test_zero_query_gives_mean_and_log_len():
+    B, H, G = 2, 3, 2
+    q = np.zeros((B, H, O.WIDTH))
+    rows = _rows(B, [7, 20], 61)
+    out, lse = O.tpla_decode_ref(q, rows, G, "replicate", SCALE)
+    for b in range(B):
+        mean = rows[b][:, :512].mean(axis=0)
+        assert np.allclose(out[b], np.tile(mean, (H, 1)), rtol=1e-12, atol=1e-13)
+        assert np.allclose(lse[b], math.log(rows[b].shape[0]), rtol=0, atol=1e-13)
+
+
+def test_empty_request():
+    q = _rand((2, 3, O.WIDTH), 71)
+    rows = _rows(2, [0, 4], 72)
+    out, lse = O.tpla_decode_ref(q, rows, 2, "replicate", SCALE)
+    assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))
+    assert np.all(np.isfinite(lse[1]))
+
+
+def test_one_shard_mode_is_a_slice():
+    B, H, G = 2, 4, 4
+    q = _rand((B, H, O.WIDTH), 81)
+    rows = _rows(B, [30, 5], 82)
+    full, lfull = O.tpla_decode_ref(q, rows, G, "split", SCALE)
+    for s in range(G):
+        one, l1 = O.tpla_decode_ref(q, rows, G, "split", SCALE, shard=s)
+        assert one.shape == (B, H, 512 // G)
+        assert np.array_equal(one, full[:, :, s * 128:(s + 1) * 128])
+        assert np.array_equal(l1[..., 0], lfull[..., s])
+
+
+def test_softmax_shift_invariance():
+    """Adding a constant to every logit of a shard (here: via a rope column
+    that is constant over tokens) leaves the output unchanged and shifts lse
+    by exactly that constant."""
+    B, H, L = 1, 2, 9
+    q = _rand((B, H, O.WIDTH), 91)
+    rows = _rows(B, [L], 92)
+    base_rows = [rows[0].copy()]
+    base_rows[0][:, 512:] = 0.0
+    shifted = [base_rows[0].copy()]
+    shifted[0][:, 512] = 3.0
+    o0, l0 = O.tpla_decode_ref(q, base_rows, 2, "replicate", SCALE)
+    o1, l1 = O.tpla_decode_ref(q, shifted, 2, "replicate", SCALE)
+    assert np.allclose(o0, o1, rtol=1e-12, atol=1e-13)
+    assert np.allclose(l1 - l0, SCALE * 3.0 * q[0][:, 512][:, None], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- paging
+
+def test_paged_equals_contiguous():
+    rng = np.random.default_rng(101)
+    B, H, Ls = 3, 2, [70, 1, 128]
+    cont = rng.standard_normal((B, 128, O.WIDTH))
+    pages = [(L + 63) // 64 for L in Ls]
+    nb = sum(pages) + 2
+    perm = rng.permutation(nb)
+    cache = rng.standard_normal((nb, 64, O.WIDTH))
+    pt = np.zeros((B, 2), dtype=np.int64)
+    off = 0
+    for b in range(B):
+        for p in range(pages[b]):
+            blk = perm[off + p]
+            pt[b, p] = blk
+            cache[blk] = cont[b, p * 64:(p + 1) * 64]
+        off += pages[b]
+    q = rng.standard_normal((B, H, O.WIDTH))
+    a = O.tpla_decode_paged_ref(q, cache, Ls, pt, 2, "replicate", SCALE)
+    c = O.tpla_decode_paged_ref(q, cont, Ls, None, 2, "replicate", SCALE)
+    assert np.array_equal(a[0], c[0]) and np.array_equal(a[1], c[1])
+
+
+# ---------------------------------------------------------------- split + merge
+
+@pytest.mark.parametrize("bounds", [[0, 5, 40], [0, 0, 13, 13, 40], [0, 1, 2, 3, 40],
+                                    [0, 40, 64]])
+def test_split_merge_equals_unsplit(bounds):
+    B, H, G = 2, 3, 2
+    q = _rand((B, H, O.WIDTH), 111)
+    rows = _rows(B, [40, 17], 112)
+    os_, ls_ = O.split_decode_ref(q, rows, G, "replicate", SCALE, bounds)
+    ou, lu = O.tpla_decode_ref(q, rows, G, "replicate", SCALE)
+    assert np.allclose(os_, ou, rtol=1e-12, atol=1e-13)
+    assert np.allclose(ls_, lu, rtol=1e-12, atol=1e-12)
+
+
+def test_lse_merge_closed_form():
+    # two chunks with lse 0 and ln 3: weights 1/4 and 3/4
+    o = np.array([[[1.0, 0.0]], [[0.0, 1.0]]])
+    l = np.array([[0.0], [math.log(3.0)]])
+    out, lse = O.lse_merge_ref(o, l)
+    assert np.allclose(out, [[0.25, 0.75]])
+    assert np.allclose(lse, [math.log(4.0)])
+    # all-empty chunks -> zero output, -inf lse
+    out, lse = O.lse_merge_ref(o, np.full((2, 1), -np.inf))
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+    # one empty chunk contributes nothing
+    out, lse = O.lse_merge_ref(o, np.array([[-np.inf], [0.5]]))
+    assert np.allclose(out, [[0.0, 1.0]]) and np.allclose(lse, [0.5])
+
+
+# ---------------------------------------------------------------- Hadamard
+
+@pytest.mark.parametrize("n", [1, 2, 8, 64, 512])
+def test_hadamard_matches_scipy_and_is_involution(n):
+    from scipy.linalg import hadamard
+    Hm = O.hadamard_matrix(n)
+    assert np.allclose(Hm, hadamard(n) / math.sqrt(n), rtol=0, atol=1e-15)
+    assert np.allclose(Hm @ Hm, np.eye(n), atol=1e-12)
+    e0 = np.zeros(n)
+    e0[0] = 1.0
+    assert np.allclose(Hm @ e0, np.full(n, 1 / math.sqrt(n)))
+
+
+def test_hadamard_kron_recursion():
+    h2 = np.array([[1.0, 1.0], [1.0, -1.0]])
+    M = np.array([[1.0]])
+    for _ in range(9):
+        M = np.kron(M, h2)
+    assert np.allclose(O.hadamard_matrix(512), M / math.sqrt(512), atol=1e-15)
+
+
+def test_hadamard_ref_leaves_rope_and_preserves_norm():
+    x = _rand((5, O.WIDTH), 121)
+    y = O.hadamard_ref(x, 512)
+    assert np.array_equal(y[:, 512:], x[:, 512:])
+    assert np.allclose(np.linalg.norm(y[:, :512], axis=1), np.linalg.norm(x[:, :512], axis=1))
+    assert np.allclose(O.hadamard_ref(y, 512), x, atol=1e-12)
+
+
+def test_hadamard_invariance_for_g1():
+    """Orthogonal U absorbed into q and the cache leaves exact MLA unchanged
+    after un-rotating the latent output (U U^T = I)."""
+    B, H = 2, 3
+    q = _rand((B, H, O.WIDTH), 131)
+    rows = _rows(B, [25, 64], 132)
+    o, l = O.tpla_decode_ref(q, rows, 1, "replicate", SCALE)
+    qr = O.hadamard_ref(q, 512)
+    rr = [O.hadamard_ref(r, 512) for r in rows]
+    o2, l2 = O.tpla_decode_ref(qr, rr, 1, "replicate", SCALE)
+    o2 = O.hadamard_ref(o2, 512)
+    assert np.allclose(o, o2, atol=1e-12)
+    assert np.allclose(l, l2, atol=1e-12)
+
+
+def test_hadamard_changes_tpla_g2():
+    """For G>1 the rotation is not absorbed exactly (the per-shard softmax is
+    an approximation): the rotated result differs from the unrotated one."""
+    B, H = 1, 2
+    q = _rand((B, H, O.WIDTH), 141)
+    rows = _rows(B, [30], 142)
+    o, _ = O.tpla_decode_ref(q, rows, 2, "replicate", SCALE)
+    o2, _ = O.tpla_decode_ref(O.hadamard_ref(q, 512), [O.hadamard_ref(rows[0], 512)],
+                              2, "replicate", SCALE)
+    assert not np.allclose(o, O.hadamard_ref(o2, 512), atol=1e-6)
+
+
+# ---------------------------------------------------------------- combine
+
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_vup_concat_equals_sum_over_shards(G):
+    out = _rand((3, 4, 512), 151)
+    W = _rand((4, 512, 128), 152)
+    assert np.allclose(O.vup_ref(out, W), O.vup_sharded_ref(out, W, G), atol=1e-10)
+
+
+def test_vup_hadamard_fold_and_bruteforce():
+    out = _rand((2, 2, 512), 161)
+    W = _rand((2, 512, 8), 162)
+    Hm = O.hadamard_matrix(512)
+    W_folded = np.einsum("ij,hjk->hik", Hm, W)
+    assert np.allclose(O.vup_ref(O.hadamard_ref(out, 512), W), O.vup_ref(out, W_folded), atol=1e-10)
+    y = O.vup_ref(out, W)
+    for b in range(2):
+        for h in range(2):
+            for k in range(8):
+                assert abs(y[b, h, k] - sum(out[b, h, j] * W[h, j, k] for j in range(512))) < 1e-10
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def test_pins_catch_planted_mistakes(monkeypatch):
+    """Plant plausible mistakes in a copy of the oracle's primitive and check
+    that an independent pin fails for each."""
+    B, H, L = 1, 2, 6
+    q = _rand((B, H, O.WIDTH), 171)
+    rows = _rows(B, [L], 172)
+    keys = rows[0].tolist()
+    vals = rows[0][:, :512].tolist()
+    ob, lb = O.attention_bruteforce(q[0].tolist(), keys, vals, SCALE)
+    good = O.attention_ref
+
+    def no_scale(qh, k, v, s):
+        return good(qh, k, v, 1.0)
+
+    def dropped_rope(qh, k, v, s):
+        kk = np.array(k, copy=True)
+        kk[:, 512:] = 0.0
+        return good(qh, kk, v, s)
+
+    def wrong_sign(qh, k, v, s):
+        return good(qh, k, v, -s)
+
+    for bad in (no_scale, dropped_rope, wrong_sign):
+        monkeypatch.setattr(O, "attention_ref", bad)
+        out, lse = O.mla_decode_ref(q, rows, SCALE)
+        assert not np.allclose(out[0], np.array(ob), atol=1e-9)
+    monkeypatch.setattr(O, "attention_ref", good)
