@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Latent-KV decode throughput of libtpla on B200.
+
+One step = one pass of the whole decode hot path over one batch of the
+DeepSeek-V3-shaped workload (B=64 requests, H=128 heads, 32768 cached
+tokens each, paged 64-token blocks, 576 bf16 values per token):
+  tpla_decode_ex (TPLA, G shards, split-KV + log-sum-exp merge inside)
+  -> tpla_vup_combine (V up-projection; stands in for the TP all-reduce).
+The Walsh-Hadamard reparameterisation is applied once to q, the cache and
+(folded) W_uv before timing, as a deployment folds it into the weights.
+
+Metric: latent-KV GB/s = algorithmic cache bytes per step / step time
+(also decode tokens/s per layer).  Inputs (2.4 GB) exceed the 126 MB L2, so
+no flush is needed between steps.  Multi-GPU runs are independent replicas
+(the path has no cross-GPU exchange on one node in this build).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_latent_kv_dim_b200.workloads import (LATENT, ROPE, WIDTH, CONFIGS,  # noqa: E402
+                                              make_workload)
+
+METRIC = "latent-KV GB/s & decode tok/s/layer at H=128 L=32K (% HBM peak), vs G"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="dsv3", choices=sorted(CONFIGS))
+    ap.add_argument("--G", type=int, default=2)
+    ap.add_argument("--rope", default="replicate", choices=["replicate", "split"])
+    ap.add_argument("--no-hadamard", action="store_true")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "generic", "sm100"])
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--no-extras", action="store_true", help="skip the per-G sweep")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops_per_token_head(G, shard=None, rope_mode="replicate"):
+    """Algorithmic MMA flops per (token, head): QK over each shard's key
+    columns plus PV over its latent columns."""
+    d = LATENT // G
+    r = ROPE if rope_mode == "replicate" else ROPE // G
+    shards = G if shard is None else 1
+    return shards * (2 * (d + r) + 2 * d)
+
+
+def decode_kernel_hash():
+    h = hashlib.sha256()
+    for f in ("decode_sm100.cu", "decode_generic.cu", "merge.cu"):
+        p = os.path.join(ROOT, "mla_latent_kv_dim_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_name, workload):
+    """Per-launch DRAM bytes of the decode kernel from a committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(kernel_name, {}).get(workload)
+        if e and e.get("source_hash") == decode_kernel_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, G, rope, hadamard, budget_s):
+    """Time the float64 oracle on whole requests of the workload until about
+    ``budget_s`` seconds have passed.  Returns (GB/s, seconds, requests)."""
+    from oracle import tpla_oracle as O  # CPU baseline leg only
+    from mla_latent_kv_dim_b200.workloads import as_f64
+    done_bytes = 0
+    t_total = 0.0
+    reqs = 0
+    b = 0
+    while t_total < budget_s and b < w.B:
+        L = int(w.seq_lens[b])
+        pages = (L + 63) // 64
+        if w.page_table is not None:
+            rows = as_f64(w.cache[w.page_table[b, :pages].long()].reshape(pages * 64, WIDTH)[:L])
+        else:
+            rows = as_f64(w.cache[b, :L])
+        q = as_f64(w.q[b:b + 1])
+        t0 = time.perf_counter()
+        if hadamard:
+            q = O.hadamard_ref(q, 512)
+            rows = O.hadamard_ref(rows, 512)
+        O.tpla_decode_ref(q, [rows], G, rope, np.float32(w.scale))
+        t_total += time.perf_counter() - t0
+        done_bytes += L * WIDTH * 2
+        reqs += 1
+        b += 1
+    return done_bytes / t_total / 1e9, t_total, reqs
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = make_workload(args.config)
+    hadamard = not args.no_hadamard
+    per_step = []
+    reqs = 0
+    for i in range(args.warmup + args.steps):
+        gbs, t, n = oracle_sample(w, args.G, args.rope, hadamard,
+                                  budget_s=max(0.5, 120.0 / (args.warmup + args.steps)))
+        if i >= args.warmup:
+            per_step.append(gbs)
+            reqs = n
+    v = statistics.mean(per_step)
+    cores = blas_threads()
+    sample = (f"{reqs} request(s) x {w.H} heads x {int(w.seq_lens[0])} tokens of the "
+              f"{args.config} workload per step, G={args.G}, float64 NumPy oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.config, "G": args.G, "rope_mode": args.rope,
+                   "hadamard": hadamard},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import mla_latent_kv_dim_b200 as tp
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    hadamard = not args.no_hadamard
+    G, rope = args.G, args.rope
+
+    w = make_workload(args.config, pin=True)
+    q = w.q.to(dev)
+    cache = w.cache.to(dev, non_blocking=True)
+    seq = w.seq_lens.to(dev)
+    pt = None if w.page_table is None else w.page_table.to(dev)
+    W = w.W_uv.to(dev) if w.W_uv is not None else None
+    if W is None:
+        g = torch.Generator().manual_seed(1234)
+        W = (0.02 * torch.randn((w.H, LATENT, 128), generator=g)).to(torch.bfloat16).to(dev)
+    if hadamard:
+        # one-off reparameterisation: q, cache and the folded V up-projection
+        tp.hadamard_apply(q, LATENT)
+        tp.hadamard_apply(cache, LATENT)
+        Wt = W.transpose(1, 2).contiguous()
+        tp.hadamard_apply(Wt, LATENT)
+        W = Wt.transpose(1, 2).contiguous()
+    torch.cuda.synchronize()
+    B, H = w.B, w.H
+    out = torch.empty((B, H, LATENT), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, H, G), dtype=torch.float32, device=dev)
+    y = torch.empty((B, H, W.shape[2]), dtype=torch.float32, device=dev)
+    need = tp.decode_workspace_size(q, cache, seq, pt, G, rope, out, num_splits=args.num_splits,
+                                    kernel=args.kernel)
+    ws = torch.empty(max(16, need), dtype=torch.uint8, device=dev)
+    bytes_step = w.latent_kv_bytes(G)
+    flops_step = float(w.seq_lens.to(torch.int64).sum()) * H * flops_per_token_head(G, None, rope)
+    stream = torch.cuda.current_stream()
+
+    def decode_once(qq, o, l, shard=None, GG=G):
+        tp.decode(qq, cache, seq, pt, GG, rope, w.scale, out=o, lse=l, shard=shard,
+                  num_splits=args.num_splits, kernel=args.kernel, workspace=ws)
+
+    def step(ev_a=None, ev_b=None):
+        if ev_a is not None:
+            ev_a.record(stream)
+        decode_once(q, out, lse)
+        if ev_b is not None:
+            ev_b.record(stream)
+        tp.vup_combine(out, W, y)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    n0 = tp.launch_count()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(*evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    n_launch = tp.launch_count() - n0
+    clk = clocks.stop()
+    if dist:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    if dist:
+        tt = torch.tensor([ms, dec_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, dec_ms = float(tt[0]), float(tt[1])
+    t_step = ms / 1e3 / args.steps
+    value = world * bytes_step / t_step / 1e9
+    tok_s = world * B / t_step
+
+    # ---- end to end through the public API: host q in, host y out
+    q_host = q.cpu().pin_memory()
+    seq_host = w.seq_lens.pin_memory()
+    pt_host = None if w.page_table is None else w.page_table.pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    q_in = torch.empty_like(q)
+
+    def e2e_step():
+        q_in.copy_(q_host, non_blocking=True)
+        seq.copy_(seq_host, non_blocking=True)
+        if pt is not None:
+            pt.copy_(pt_host, non_blocking=True)
+        decode_once(q_in, out, lse)
+        tp.vup_combine(out, W, y)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if dist:
+        tt = torch.tensor([e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e_ms = float(tt[0])
+    e2e_val = world * bytes_step / (e_ms / 1e3 / args.steps) / 1e9
+    h2d = q.numel() * 2 + seq.numel() * 4 + (pt.numel() * 4 if pt is not None else 0)
+    d2h = y.numel() * 4
+
+    # ---- roofline of the dominant kernel (decode), live CUDA-event timing
+    dec_s = dec_ms / 1e3
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tc_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    achieved_gbs = bytes_step / dec_s / 1e9
+    achieved_tf = flops_step / dec_s / 1e12
+    t_hbm = bytes_step / (hbm_peak * 1e9)
+    t_tc = flops_step / (tc_peak * 1e12)
+    used = "sm100" if args.kernel != "generic" and _sm100_used(tp, q, cache, seq, pt, G, rope, out,
+                                                                args) else "generic"
+    kname = "tpla_decode_sm100" if used == "sm100" else "decode_generic_kernel"
+    traffic = recorded_traffic(kname, args.config)
+    if t_tc > t_hbm:
+        roof = {"bound": "tensor", "achieved": round(achieved_tf, 2), "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(achieved_tf / tc_peak, 4)}
+    else:
+        roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(achieved_gbs / hbm_peak, 4)}
+    roof.update({"traffic": traffic, "kernel": kname,
+                 "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
+                 "hbm_gbs": round(achieved_gbs, 1), "hbm_frac": round(achieved_gbs / hbm_peak, 4),
+                 "tensor_tflops": round(achieved_tf, 2),
+                 "tensor_frac_sustained": round(achieved_tf / tc_peak, 4),
+                 "bytes_per_launch": bytes_step, "flops_per_launch": flops_step,
+                 "decode_ms": round(dec_ms, 4)})
+
+    # ---- per-G decode-only sweep (vs G), full and one-shard
+    vs_G = []
+    if not args.no_extras:
+        for GG, shard in ((1, None), (2, None), (4, None), (2, 0), (4, 0)):
+            width = LATENT if shard is None else LATENT // GG
+            o2 = torch.empty((B, H, width), dtype=torch.float32, device=dev)
+            l2 = torch.empty((B, H, GG if shard is None else 1), dtype=torch.float32, device=dev)
+            for _ in range(3):
+                decode_once(q, o2, l2, shard, GG)
+            a = torch.cuda.Event(enable_timing=True)
+            bb = torch.cuda.Event(enable_timing=True)
+            n = 10
+            a.record(stream)
+            for _ in range(n):
+                decode_once(q, o2, l2, shard, GG)
+            bb.record(stream)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(bb) / 1e3 / n
+            nb = w.latent_kv_bytes(GG, shard, rope)
+            vs_G.append({"G": GG, "mode": "full" if shard is None else "one-shard",
+                         "bytes": nb, "decode_us": round(t * 1e6, 1),
+                         "GB_s": round(nb / t / 1e9, 1),
+                         "hbm_frac": round(nb / t / 1e9 / hbm_peak, 4),
+                         "tok_s_layer": round(B / t, 1)})
+            del o2, l2
+
+    cpu = None
+    if rank == 0 and world == 1:
+        torch.cuda.synchronize()
+        gbs, secs, reqs = oracle_sample(w, G, rope, hadamard, args.cpu_seconds)
+        cpu = {"value": round(gbs, 5), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{reqs} whole request(s) x {H} heads x {int(w.seq_lens[0])} tokens, "
+                         f"G={G}, {'Hadamard, ' if hadamard else ''}{secs:.1f} s of float64 NumPy"}
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; no checkpoints or datasets)",
+        "config": {"workload": args.config, "B": B, "H": H,
+                   "seq_len": int(w.seq_lens.max()), "G": G, "rope_mode": rope,
+                   "hadamard": hadamard, "paged_block": 64, "kernel": used,
+                   "num_splits": args.num_splits or "auto",
+                   "step": "decode (+LSE merge) + V-up combine",
+                   "l2": "inputs 2.4 GB > 126 MB L2; no flush needed",
+                   "parallelism": f"replicas x{world}"},
+        "tok_s_layer": round(tok_s, 1),
+        "hbm_frac_step": round(value / world / hbm_peak, 4),
+        "roofline": roof, "vs_G": vs_G, "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms / args.steps, 4)},
+        "gpu_launches": n_launch, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _sm100_used(tp, q, cache, seq, pt, G, rope, out, args):
+    try:
+        tp.decode_workspace_size(q, cache, seq, pt, G, rope, out, kernel="sm100")
+        return True
+    except tp.TplaError:
+        return False
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,222 @@
+/*
+ * tpla.h -- C ABI of libtpla: single-token MLA decode attention over the
+ * compressed latent KV cache (absorbed form) and its TPLA variant, on
+ * NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources: the GitHub feature request "Bandwidth-optimal
+ * tensor-parallel sharding of MLA (latent-cache sharding / TPLA)", sections
+ * "Background / problem" and "Directions under investigation"; the TPLA
+ * abstract; the pith.science review of arXiv 2508.15881, key machinery and
+ * skeptic critique of Eq. 6):
+ *
+ *   Each cached token holds 576 values: 512 latent (c_KV) + 64 rope key.
+ *   For request b, head h and shard g (G shards; d = 512 / G):
+ *     s_t   = scale * ( q[b,h,I_g] . c_t[I_g]  +  q[b,h,R_g] . c_t[R_g] )
+ *     out[b,h,I_g] = sum_t softmax_t(s) * c_t[I_g]
+ *     lse[b,h,g]   = ln sum_t exp(s_t)
+ *   I_g = [g*d, (g+1)*d).  R_g = all 64 rope columns (rope_mode REPLICATE)
+ *   or the contiguous slice [512 + g*64/G, 512 + (g+1)*64/G) (SPLIT).
+ *   G = 1 is exact MLA decode.  G > 1 is TPLA: every shard runs its own,
+ *   unscaled softmax; shard outputs are laid side by side in latent space
+ *   and later summed through the V up-projection (tpla_vup_combine), which
+ *   stands in for the tensor-parallel all-reduce.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are described by tpla_tensor: data pointer, dtype, rank and
+ *     per-dimension sizes and strides (strides in ELEMENTS).  The innermost
+ *     dimension must be contiguous (stride 1).
+ *   - All tensor data lives in device memory of the current CUDA device and
+ *     is owned by the caller.  The library never frees or retains pointers.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream)
+ *     and performs no host synchronisation, except tpla_get_device_status.
+ *   - Inputs are never modified, except the buffer of tpla_hadamard_apply.
+ *   - Return value: TPLA_OK (0) or a negative tpla_status.  Arguments are
+ *     validated before anything is launched; on an argument error nothing is
+ *     launched and no memory is touched.  No C++ exception crosses the ABI.
+ */
+#ifndef TPLA_H
+#define TPLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TPLA_VERSION 100
+
+#if defined(__GNUC__)
+#define TPLA_API __attribute__((visibility("default")))
+#else
+#define TPLA_API
+#endif
+
+/* cudaStream_t without including CUDA headers. */
+typedef struct CUstream_st* tpla_stream_t;
+
+enum tpla_dtype { TPLA_BF16 = 1, TPLA_F32 = 2, TPLA_I32 = 3 };
+
+enum tpla_status {
+  TPLA_OK = 0,
+  TPLA_ERR_INVALID_ARG = -1,   /* null pointer, shape/stride/dtype mismatch  */
+  TPLA_ERR_UNSUPPORTED = -2,   /* valid request this build cannot run        */
+  TPLA_ERR_CUDA = -3,          /* a CUDA call failed; see tpla_last_cuda_error */
+  TPLA_ERR_WORKSPACE = -4,     /* workspace missing or too small             */
+  TPLA_ERR_DEVICE_TIMEOUT = -5,/* a kernel gave up waiting (device status)   */
+  TPLA_ERR_DEVICE_BOUNDS = -6  /* a kernel met an out-of-range page id or
+                                  sequence length (device status)            */
+};
+
+enum tpla_rope_mode { TPLA_ROPE_REPLICATE = 0, TPLA_ROPE_SPLIT = 1 };
+
+enum tpla_kernel_choice {
+  TPLA_KERNEL_AUTO = 0,     /* tensor-core kernel where the shape allows it   */
+  TPLA_KERNEL_GENERIC = 1,  /* portable CUDA-core kernel (any supported shape) */
+  TPLA_KERNEL_SM100 = 2     /* tcgen05/TMA kernel; UNSUPPORTED if it cannot   */
+};
+
+typedef struct {
+  void* data;
+  int32_t dtype;     /* enum tpla_dtype */
+  int32_t ndim;      /* 1..4 */
+  int64_t shape[4];
+  int64_t stride[4]; /* elements */
+} tpla_tensor;
+
+typedef struct {
+  /* 0 = automatic split of the KV sequence (balanced over the GPU's SMs);
+     k >= 1 = cut every request's tokens into k equal chunks and merge them
+     with the log-sum-exp rule.  1 = no split. */
+  int32_t num_splits;
+  /* -1 = compute all G shards.  s in [0, G) = one-shard mode: read only the
+     columns shard s needs (the bytes one tensor-parallel rank reads) and
+     write out [B, H, d], lse [B, H, 1]. */
+  int32_t shard;
+  int32_t kernel;    /* enum tpla_kernel_choice */
+  int32_t reserved;  /* must be 0 */
+  /* Device scratch for split partial results; see
+     tpla_decode_workspace_size.  May be NULL when the size is 0. */
+  void* workspace;
+  size_t workspace_bytes;
+} tpla_decode_opts;
+
+/*
+ * tpla_decode_ex -- latent-KV decode attention, MLA (G = 1) or TPLA (G > 1).
+ *
+ *   q          [B, H, 576] bf16.  Query in absorbed form (q_nope already
+ *              multiplied by W_UK, then rope query).  Rows must start on
+ *              16-byte boundaries (stride[1] % 8 == 0, data 16-byte aligned).
+ *   kv_cache   paged:      [num_blocks, 64, 576] bf16 (64-token pages),
+ *              contiguous: [B, Lmax, 576] bf16 when page_table is NULL.
+ *              stride[1] % 8 == 0, stride[0] % 8 == 0, 16-byte aligned.
+ *   seq_lens   [B] int32: tokens of each request (0 allowed).
+ *   page_table [B, max_pages] int32 or NULL.  Entry p of row b is the
+ *              physical block holding tokens [64p, 64p + 64) of request b;
+ *              only entries p < ceil(seq_lens[b] / 64) are read.
+ *   G          1, 2, 4 or 8 latent shards.
+ *   rope_mode  TPLA_ROPE_REPLICATE or TPLA_ROPE_SPLIT.
+ *   scale      softmax scale applied to the dot products (finite).
+ *   out        [B, H, 512] (or [B, H, d] in one-shard mode), f32 or bf16.
+ *   lse        NULL or [B, H, G] (one-shard: [B, H, 1]) f32, natural log.
+ *   opts       NULL = defaults {0, -1, AUTO, 0, NULL, 0}.
+ *
+ * A request with seq_lens = 0 gets out = 0 and lse = -inf.  Page ids outside
+ * [0, num_blocks) or seq_lens larger than the cache can hold are not read;
+ * the kernel records TPLA_ERR_DEVICE_BOUNDS in the device status word
+ * (tpla_get_device_status) and treats the missing tokens as absent.
+ */
+TPLA_API int tpla_decode_ex(const tpla_tensor* q, const tpla_tensor* kv_cache,
+                   const tpla_tensor* seq_lens, const tpla_tensor* page_table,
+                   int G, int rope_mode, float scale,
+                   tpla_tensor* out, tpla_tensor* lse,
+                   const tpla_decode_opts* opts, tpla_stream_t stream);
+
+/*
+ * tpla_decode_workspace_size -- bytes of device workspace tpla_decode_ex
+ * needs for these arguments and options (0 when no split is used).  Same
+ * validation as tpla_decode_ex; writes the size to *bytes.
+ */
+TPLA_API int tpla_decode_workspace_size(const tpla_tensor* q, const tpla_tensor* kv_cache,
+                               const tpla_tensor* seq_lens,
+                               const tpla_tensor* page_table, int G,
+                               int rope_mode, const tpla_tensor* out,
+                               const tpla_decode_opts* opts, size_t* bytes);
+
+/*
+ * tpla_decode -- tpla_decode_ex with default options.  When a split is used
+ * the workspace comes from the stream-ordered allocator (cudaMallocAsync /
+ * cudaFreeAsync on `stream`), so this convenience call allocates; callers
+ * that manage memory themselves use tpla_decode_ex.
+ */
+TPLA_API int tpla_decode(const tpla_tensor* q, const tpla_tensor* kv_cache,
+                const tpla_tensor* seq_lens, const tpla_tensor* page_table,
+                int G, int rope_mode, float scale, tpla_tensor* out,
+                tpla_tensor* lse, tpla_stream_t stream);
+
+/*
+ * tpla_lse_merge -- exact merge of S partial attention results over disjoint
+ * key chunks (the log-sum-exp rule of the sequence-split alternative in the
+ * feature request's "Directions under investigation").
+ *   o_parts   [S, B, H, Wd] f32, each chunk's normalised output.
+ *   lse_parts [S, B, H, Gs] f32; Wd must be a multiple of Gs and shard k of
+ *             a row owns columns [k*Wd/Gs, (k+1)*Wd/Gs).
+ *   out       [B, H, Wd] f32 or bf16;  lse NULL or [B, H, Gs] f32.
+ * lse = ln sum_s exp(lse_s); out = sum_s exp(lse_s - lse) o_s.  Chunks with
+ * lse = -inf contribute nothing; if every chunk is -inf, out = 0, lse = -inf.
+ */
+TPLA_API int tpla_lse_merge(const tpla_tensor* o_parts, const tpla_tensor* lse_parts,
+                   tpla_tensor* out, tpla_tensor* lse, tpla_stream_t stream);
+
+/*
+ * tpla_hadamard_apply -- in-place orthonormal Walsh-Hadamard transform of
+ * the first `dim` columns of every row of `buf` (Sylvester / natural order,
+ * entries (-1)^popcount(i & j) / sqrt(dim)); other columns are untouched.
+ * The transform is its own inverse.  The orthogonal reparameterisation
+ * applied before slicing (feature request, "Directions under investigation";
+ * TPLA abstract).
+ *   buf  bf16 or f32, ndim 1..4, innermost dimension >= dim and contiguous;
+ *        every other dimension indexes rows.
+ *   dim  power of two in [32, 1024].
+ * Arithmetic is f32; bf16 rows are rounded once on store.
+ */
+TPLA_API int tpla_hadamard_apply(tpla_tensor* buf, int dim, tpla_stream_t stream);
+
+/*
+ * tpla_vup_combine -- y[b, h, :] = sum_j out_latent[b, h, j] * W_uv[h, j, :].
+ * The V up-projection; with shard outputs laid side by side in latent space,
+ * the contraction over j is the sum over shards that the tensor-parallel
+ * all-reduce performs (feature request, "Directions under investigation").
+ *   out_latent [B, H, 512] f32 or bf16;  W_uv [H, 512, Dv] bf16, Dv a
+ *   multiple of 16 and <= 256;  y [B, H, Dv] f32.
+ * Accumulation is f32 on tensor cores; an f32 out_latent is split into two
+ * bf16 terms (hi + lo) so that its rounding does not limit accuracy.
+ */
+TPLA_API int tpla_vup_combine(const tpla_tensor* out_latent, const tpla_tensor* W_uv,
+                     tpla_tensor* y, tpla_stream_t stream);
+
+/* Human-readable name of a tpla_status code (static string). */
+TPLA_API const char* tpla_error_string(int status);
+
+/* The cudaError_t of the most recent TPLA_ERR_CUDA on this host thread. */
+TPLA_API int tpla_last_cuda_error(void);
+
+/*
+ * tpla_get_device_status -- synchronise `stream`, then read and clear the
+ * status word the kernels of this library set on the current device
+ * (TPLA_OK, TPLA_ERR_DEVICE_BOUNDS or TPLA_ERR_DEVICE_TIMEOUT).
+ */
+TPLA_API int tpla_get_device_status(tpla_stream_t stream, int* status);
+
+/* Number of CUDA kernels this library has launched in this process (all
+ * devices, all host threads).  Lets a caller count the library's launches
+ * inside a timed region. */
+TPLA_API int64_t tpla_launch_count(void);
+
+/* TPLA_VERSION of the loaded library. */
+TPLA_API int tpla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TPLA_H */

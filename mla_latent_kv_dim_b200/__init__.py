@@ -1,0 +1,13 @@
+"""B200-native MLA latent-KV decode and TPLA (Tensor-Parallel Latent Attention).
+
+The compute lives in ``libtpla.so`` (C ABI, include/tpla.h): hand-written
+CUDA kernels for sm_100a.  This package holds the ctypes binding
+(``_native``), the in-tree build (``build``) and the seeded synthetic
+workloads (``workloads``).
+"""
+from ._native import (TplaError, decode, decode_simple, decode_workspace_size,  # noqa: F401
+                      device_status, error_string, hadamard_apply, launch_count, lse_merge, lib,
+                      version, vup_combine)
+
+__all__ = ["TplaError", "decode", "decode_simple", "decode_workspace_size", "device_status",
+           "error_string", "hadamard_apply", "launch_count", "lse_merge", "lib", "version", "vup_combine"]

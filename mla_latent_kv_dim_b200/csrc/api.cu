@@ -1,0 +1,349 @@
+// libtpla C ABI: argument validation, kernel selection, errors, status.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "internal.h"
+#include "tpla.h"
+
+namespace tpla {
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+std::atomic<int64_t> g_launches{0};
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = (int)e;
+  return TPLA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool check_tensor(const tpla_tensor* t, int dtype, int ndim) {
+  if (!t || t->dtype != dtype || t->ndim != ndim) return false;
+  for (int i = 0; i < ndim; ++i) {
+    if (t->shape[i] < 0) return false;
+    if (t->stride[i] < 0) return false;
+  }
+  if (ndim > 0 && t->shape[ndim - 1] > 1 && t->stride[ndim - 1] != 1) return false;
+  bool empty = false;
+  for (int i = 0; i < ndim; ++i) empty |= t->shape[i] == 0;
+  if (!empty && !t->data) return false;
+  return true;
+}
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+
+// Flatten and validate a decode call.
+int build_problem(const tpla_tensor* q, const tpla_tensor* kv, const tpla_tensor* seq,
+                  const tpla_tensor* pt, int G, int rope_mode, float scale,
+                  const tpla_tensor* out, const tpla_tensor* lse,
+                  const tpla_decode_opts* opts, DecodeProblem* p) {
+  if (!q || !kv || !seq || !out) return TPLA_ERR_INVALID_ARG;
+  if (!(G == 1 || G == 2 || G == 4 || G == 8)) return TPLA_ERR_INVALID_ARG;
+  if (rope_mode != TPLA_ROPE_REPLICATE && rope_mode != TPLA_ROPE_SPLIT) return TPLA_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return TPLA_ERR_INVALID_ARG;
+  int shard = opts ? opts->shard : -1;
+  if (shard < -1 || shard >= G) return TPLA_ERR_INVALID_ARG;
+  if (opts && (opts->reserved != 0 || opts->num_splits < 0)) return TPLA_ERR_INVALID_ARG;
+  if (opts && (opts->kernel < TPLA_KERNEL_AUTO || opts->kernel > TPLA_KERNEL_SM100))
+    return TPLA_ERR_INVALID_ARG;
+
+  if (!check_tensor(q, TPLA_BF16, 3) || q->shape[2] != kWidth) return TPLA_ERR_INVALID_ARG;
+  const int64_t B = q->shape[0], H = q->shape[1];
+  if (B > (1 << 20) || H > 4096) return TPLA_ERR_UNSUPPORTED;
+  if (!check_tensor(seq, TPLA_I32, 1) || seq->shape[0] != B) return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(kv, TPLA_BF16, 3) || kv->shape[2] != kWidth) return TPLA_ERR_INVALID_ARG;
+  const bool paged = pt != nullptr;
+  if (paged) {
+    if (!check_tensor(pt, TPLA_I32, 2) || pt->shape[0] != B) return TPLA_ERR_INVALID_ARG;
+    if (kv->shape[1] != kBlock) return TPLA_ERR_UNSUPPORTED;  // 64-token pages only
+    if (pt->shape[1] < 1 && B > 0) return TPLA_ERR_INVALID_ARG;
+    if (pt->shape[1] > (1 << 24)) return TPLA_ERR_UNSUPPORTED;
+  } else {
+    if (kv->shape[0] != B) return TPLA_ERR_INVALID_ARG;
+  }
+  // 16-byte rows (TMA and vector loads)
+  if (B > 0 && H > 0) {
+    if (!aligned16(q->data) || (q->stride[1] % 8) || (q->stride[0] % 8)) return TPLA_ERR_INVALID_ARG;
+  }
+  if (kv->shape[0] > 0 && kv->shape[1] > 0) {
+    if (!aligned16(kv->data) || (kv->stride[1] % 8) || (kv->stride[0] % 8)) return TPLA_ERR_INVALID_ARG;
+  }
+
+  const int n_shards = shard < 0 ? G : 1;
+  const int width = shard < 0 ? kLatent : kLatent / G;
+  if (!out || (out->dtype != TPLA_F32 && out->dtype != TPLA_BF16)) return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(out, out->dtype, 3) || out->shape[0] != B || out->shape[1] != H ||
+      out->shape[2] != width)
+    return TPLA_ERR_INVALID_ARG;
+  if (lse) {
+    if (!check_tensor(lse, TPLA_F32, 3) || lse->shape[0] != B || lse->shape[1] != H ||
+        lse->shape[2] != n_shards)
+      return TPLA_ERR_INVALID_ARG;
+  }
+
+  memset(p, 0, sizeof(*p));
+  p->q = q->data;
+  p->q_sb = q->stride[0];
+  p->q_sh = q->stride[1];
+  p->cache = kv->data;
+  p->c_s0 = kv->stride[0];
+  p->c_s1 = kv->stride[1];
+  p->seq_lens = reinterpret_cast<const int*>(seq->data);
+  if (paged) {
+    p->page_table = reinterpret_cast<const int*>(pt->data);
+    p->pt_sb = pt->stride[0];
+    p->max_pages = (int)pt->shape[1];
+    p->num_blocks = kv->shape[0];
+    p->cache_rows = (int64_t)pt->shape[1] * kBlock;
+  } else {
+    p->page_table = nullptr;
+    p->num_blocks = 0;
+    p->cache_rows = kv->shape[1];
+  }
+  p->B = (int)B;
+  p->H = (int)H;
+  p->G = G;
+  p->rope_mode = rope_mode;
+  p->shard = shard;
+  p->n_shards = n_shards;
+  p->out_width = width;
+  p->scale = scale;
+  p->out = out->data;
+  p->out_bf16 = out->dtype == TPLA_BF16;
+  p->o_sb = out->stride[0];
+  p->o_sh = out->stride[1];
+  p->lse = lse ? reinterpret_cast<float*>(lse->data) : nullptr;
+  p->l_sb = lse ? lse->stride[0] : 0;
+  p->l_sh = lse ? lse->stride[1] : 0;
+  return TPLA_OK;
+}
+
+enum class Path { Generic, Sm100 };
+
+int choose_path(const DecodeProblem& p, const tpla_decode_opts* opts, Path* path) {
+  int choice = opts ? opts->kernel : TPLA_KERNEL_AUTO;
+  int dev = current_device();
+  bool fast = sm100_supported(p, dev);
+  if (choice == TPLA_KERNEL_GENERIC) {
+    *path = Path::Generic;
+  } else if (choice == TPLA_KERNEL_SM100) {
+    if (!fast) return TPLA_ERR_UNSUPPORTED;
+    *path = Path::Sm100;
+  } else {
+    *path = fast ? Path::Sm100 : Path::Generic;
+  }
+  return TPLA_OK;
+}
+
+// Generic-path split count: the caller's, else enough CTAs to fill the GPU.
+int generic_splits(const DecodeProblem& p, const tpla_decode_opts* opts) {
+  int s = opts ? opts->num_splits : 0;
+  if (s >= 1) return s;
+  int64_t ctas = (int64_t)((p.H + 15) / 16) * p.B * p.n_shards;
+  int64_t want = (2 * 148 + ctas - 1) / (ctas > 0 ? ctas : 1);
+  int64_t tiles = (p.cache_rows + 255) / 256;  // at least 256 tokens per chunk
+  if (want > tiles) want = tiles;
+  if (want < 1) want = 1;
+  if (want > 64) want = 64;
+  return (int)want;
+}
+
+int workspace_needed(const DecodeProblem& p, const tpla_decode_opts* opts, Path path,
+                     size_t* bytes) {
+  if (path == Path::Generic) {
+    *bytes = generic_workspace_bytes(p, generic_splits(p, opts));
+  } else {
+    *bytes = sm100_workspace_bytes(p, opts ? opts->num_splits : 0, current_device());
+  }
+  return TPLA_OK;
+}
+
+int run_decode(const DecodeProblem& p, const tpla_decode_opts* opts, Path path, void* ws,
+               size_t ws_bytes, cudaStream_t stream) {
+  cudaError_t e;
+  if (path == Path::Generic) {
+    e = launch_decode_generic(p, generic_splits(p, opts), ws, stream);
+  } else {
+    e = launch_decode_sm100(p, opts ? opts->num_splits : 0, ws, ws_bytes, stream);
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TPLA_OK;
+}
+
+}  // namespace
+
+void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+}  // namespace tpla
+
+using namespace tpla;
+
+extern "C" {
+
+int tpla_decode_workspace_size(const tpla_tensor* q, const tpla_tensor* kv_cache,
+                               const tpla_tensor* seq_lens, const tpla_tensor* page_table,
+                               int G, int rope_mode, const tpla_tensor* out,
+                               const tpla_decode_opts* opts, size_t* bytes) {
+  if (!bytes) return TPLA_ERR_INVALID_ARG;
+  DecodeProblem p;
+  int rc = build_problem(q, kv_cache, seq_lens, page_table, G, rope_mode, 1.0f, out, nullptr,
+                         opts, &p);
+  if (rc != TPLA_OK) return rc;
+  Path path;
+  rc = choose_path(p, opts, &path);
+  if (rc != TPLA_OK) return rc;
+  return workspace_needed(p, opts, path, bytes);
+}
+
+int tpla_decode_ex(const tpla_tensor* q, const tpla_tensor* kv_cache,
+                   const tpla_tensor* seq_lens, const tpla_tensor* page_table, int G,
+                   int rope_mode, float scale, tpla_tensor* out, tpla_tensor* lse,
+                   const tpla_decode_opts* opts, tpla_stream_t stream) {
+  DecodeProblem p;
+  int rc = build_problem(q, kv_cache, seq_lens, page_table, G, rope_mode, scale, out, lse,
+                         opts, &p);
+  if (rc != TPLA_OK) return rc;
+  if (p.B == 0 || p.H == 0) return TPLA_OK;
+  Path path;
+  rc = choose_path(p, opts, &path);
+  if (rc != TPLA_OK) return rc;
+  size_t need = 0;
+  workspace_needed(p, opts, path, &need);
+  void* ws = opts ? opts->workspace : nullptr;
+  size_t have = opts ? opts->workspace_bytes : 0;
+  if (need > 0 && (!ws || have < need || !aligned16(ws))) return TPLA_ERR_WORKSPACE;
+  return run_decode(p, opts, path, ws, have, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int tpla_decode(const tpla_tensor* q, const tpla_tensor* kv_cache, const tpla_tensor* seq_lens,
+                const tpla_tensor* page_table, int G, int rope_mode, float scale,
+                tpla_tensor* out, tpla_tensor* lse, tpla_stream_t stream) {
+  DecodeProblem p;
+  int rc = build_problem(q, kv_cache, seq_lens, page_table, G, rope_mode, scale, out, lse,
+                         nullptr, &p);
+  if (rc != TPLA_OK) return rc;
+  if (p.B == 0 || p.H == 0) return TPLA_OK;
+  Path path;
+  rc = choose_path(p, nullptr, &path);
+  if (rc != TPLA_OK) return rc;
+  size_t need = 0;
+  workspace_needed(p, nullptr, path, &need);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  if (need > 0) {
+    cudaError_t e = cudaMallocAsync(&ws, need, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  rc = run_decode(p, nullptr, path, ws, need, s);
+  if (ws) {
+    cudaError_t e = cudaFreeAsync(ws, s);
+    if (rc == TPLA_OK && e != cudaSuccess) rc = cuda_fail(e);
+  }
+  return rc;
+}
+
+int tpla_lse_merge(const tpla_tensor* o_parts, const tpla_tensor* lse_parts, tpla_tensor* out,
+                   tpla_tensor* lse, tpla_stream_t stream) {
+  if (!check_tensor(o_parts, TPLA_F32, 4) || !check_tensor(lse_parts, TPLA_F32, 4))
+    return TPLA_ERR_INVALID_ARG;
+  const int64_t S = o_parts->shape[0], B = o_parts->shape[1], H = o_parts->shape[2],
+                Wd = o_parts->shape[3];
+  const int64_t Gs = lse_parts->shape[3];
+  if (lse_parts->shape[0] != S || lse_parts->shape[1] != B || lse_parts->shape[2] != H)
+    return TPLA_ERR_INVALID_ARG;
+  if (Gs < 1 || Wd % Gs != 0 || S < 1) return TPLA_ERR_INVALID_ARG;
+  if (S > 1024) return TPLA_ERR_UNSUPPORTED;
+  if (!out || (out->dtype != TPLA_F32 && out->dtype != TPLA_BF16) ||
+      !check_tensor(out, out->dtype, 3) || out->shape[0] != B || out->shape[1] != H ||
+      out->shape[2] != Wd)
+    return TPLA_ERR_INVALID_ARG;
+  if (lse && (!check_tensor(lse, TPLA_F32, 3) || lse->shape[0] != B || lse->shape[1] != H ||
+              lse->shape[2] != Gs))
+    return TPLA_ERR_INVALID_ARG;
+  cudaError_t e = launch_lse_merge(
+      reinterpret_cast<const float*>(o_parts->data),
+      reinterpret_cast<const float*>(lse_parts->data), (int)S, o_parts->stride[0],
+      lse_parts->stride[0], (int)B, (int)H, (int)Wd, (int)Gs, o_parts->stride[1],
+      o_parts->stride[2], lse_parts->stride[1], lse_parts->stride[2], out->data,
+      out->dtype == TPLA_BF16, out->stride[0], out->stride[1],
+      lse ? reinterpret_cast<float*>(lse->data) : nullptr, lse ? lse->stride[0] : 0,
+      lse ? lse->stride[1] : 0, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
+}
+
+int tpla_hadamard_apply(tpla_tensor* buf, int dim, tpla_stream_t stream) {
+  if (!buf || (buf->dtype != TPLA_BF16 && buf->dtype != TPLA_F32)) return TPLA_ERR_INVALID_ARG;
+  if (buf->ndim < 1 || buf->ndim > 4 || !check_tensor(buf, buf->dtype, buf->ndim))
+    return TPLA_ERR_INVALID_ARG;
+  if (dim < 32 || dim > 1024 || (dim & (dim - 1))) return TPLA_ERR_UNSUPPORTED;
+  if (buf->shape[buf->ndim - 1] < dim) return TPLA_ERR_INVALID_ARG;
+  if (buf->ndim > 4) return TPLA_ERR_UNSUPPORTED;
+  // rows may be described by at most three dimensions
+  cudaError_t e = launch_hadamard(buf->data, buf->dtype == TPLA_BF16, buf->ndim, buf->shape,
+                                  buf->stride, dim, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
+}
+
+int tpla_vup_combine(const tpla_tensor* out_latent, const tpla_tensor* W_uv, tpla_tensor* y,
+                     tpla_stream_t stream) {
+  if (!out_latent || (out_latent->dtype != TPLA_F32 && out_latent->dtype != TPLA_BF16))
+    return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(out_latent, out_latent->dtype, 3) || out_latent->shape[2] != kLatent)
+    return TPLA_ERR_INVALID_ARG;
+  const int64_t B = out_latent->shape[0], H = out_latent->shape[1];
+  if (!check_tensor(W_uv, TPLA_BF16, 3) || W_uv->shape[0] != H || W_uv->shape[1] != kLatent)
+    return TPLA_ERR_INVALID_ARG;
+  const int64_t Dv = W_uv->shape[2];
+  if (Dv % 16 != 0 || Dv < 16 || Dv > 256) return TPLA_ERR_UNSUPPORTED;
+  if (!check_tensor(y, TPLA_F32, 3) || y->shape[0] != B || y->shape[1] != H || y->shape[2] != Dv)
+    return TPLA_ERR_INVALID_ARG;
+  if (H > 65535) return TPLA_ERR_UNSUPPORTED;
+  cudaError_t e = launch_vup(out_latent->data, out_latent->dtype == TPLA_BF16,
+                             out_latent->stride[0], out_latent->stride[1], W_uv->data,
+                             W_uv->stride[0], W_uv->stride[1],
+                             reinterpret_cast<float*>(y->data), y->stride[0], y->stride[1],
+                             (int)B, (int)H, (int)Dv, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
+}
+
+const char* tpla_error_string(int status) {
+  switch (status) {
+    case TPLA_OK: return "ok";
+    case TPLA_ERR_INVALID_ARG: return "invalid argument";
+    case TPLA_ERR_UNSUPPORTED: return "unsupported by this build";
+    case TPLA_ERR_CUDA: return "CUDA error";
+    case TPLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case TPLA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case TPLA_ERR_DEVICE_BOUNDS: return "page id or sequence length out of range";
+    default: return "unknown status";
+  }
+}
+
+int tpla_last_cuda_error(void) { return t_last_cuda_error; }
+
+int tpla_get_device_status(tpla_stream_t stream, int* status) {
+  if (!status) return TPLA_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  int a = 0, b = 0;
+  e = status_read_clear_generic(&a);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = status_read_clear_sm100(&b);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *status = a != 0 ? a : b;
+  return TPLA_OK;
+}
+
+int tpla_version(void) { return TPLA_VERSION; }
+
+int64_t tpla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,87 @@
+// Host-side declarations shared by the libtpla translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "tpla.h"
+
+namespace tpla {
+
+constexpr int kLatent = 512;  // latent columns of a cache row
+constexpr int kRope = 64;     // rope columns of a cache row
+constexpr int kWidth = 576;   // values per cached token
+constexpr int kBlock = 64;    // tokens per cache page
+
+// One validated decode call, flattened to raw pointers and element strides.
+struct DecodeProblem {
+  const void* q;           // bf16 [B, H, 576]
+  int64_t q_sb, q_sh;
+  const void* cache;       // bf16 paged [NB, 64, 576] or contiguous [B, Lmax, 576]
+  int64_t c_s0, c_s1;      // paged: block, row strides; contiguous: batch, row
+  int64_t num_blocks;      // paged only
+  int64_t cache_rows;      // contiguous: Lmax;  paged: max_pages * 64
+  const int* seq_lens;     // [B]
+  const int* page_table;   // [B, max_pages] or nullptr (contiguous)
+  int64_t pt_sb;
+  int max_pages;
+  int B, H, G, rope_mode, shard;  // shard -1 = all shards
+  int n_shards;            // shards computed by this call: G or 1
+  int out_width;           // 512 (all shards) or 512 / G (one shard)
+  float scale;
+  void* out;               // [B, H, out_width]
+  int out_bf16;
+  int64_t o_sb, o_sh;
+  float* lse;              // [B, H, n_shards] or nullptr
+  int64_t l_sb, l_sh;
+};
+
+// Per-launch description of split partial results kept in the workspace.
+struct SplitParts {
+  float* o;     // [S, B, H, out_width]
+  float* lse;   // [S, B, H, n_shards]
+  int S;
+};
+
+// ---------------------------------------------------------------- generic path
+size_t generic_workspace_bytes(const DecodeProblem& p, int splits);
+cudaError_t launch_decode_generic(const DecodeProblem& p, int splits, void* ws,
+                                  cudaStream_t stream);
+
+// ---------------------------------------------------------------- sm100 path
+// Returns true when the tcgen05 kernel can run this problem on this device.
+bool sm100_supported(const DecodeProblem& p, int device);
+size_t sm100_workspace_bytes(const DecodeProblem& p, int num_splits, int device);
+cudaError_t launch_decode_sm100(const DecodeProblem& p, int num_splits, void* ws,
+                                size_t ws_bytes, cudaStream_t stream);
+
+// ---------------------------------------------------------------- merge
+// out[b,h,:] / lse[b,h,:] from S partials laid out as SplitParts.
+cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int S,
+                             int64_t part_stride_o, int64_t part_stride_l,
+                             int B, int H, int Wd, int Gs,
+                             int64_t po_sb, int64_t po_sh, int64_t pl_sb, int64_t pl_sh,
+                             void* out, int out_bf16, int64_t o_sb, int64_t o_sh,
+                             float* lse, int64_t l_sb, int64_t l_sh,
+                             cudaStream_t stream);
+
+// ---------------------------------------------------------------- hadamard / vup
+cudaError_t launch_hadamard(void* buf, int bf16, int ndim, const int64_t* shape,
+                            const int64_t* stride, int dim, cudaStream_t stream);
+cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64_t o_sh,
+                       const void* W, int64_t w_sh, int64_t w_sj, float* y,
+                       int64_t y_sb, int64_t y_sh, int B, int H, int Dv,
+                       cudaStream_t stream);
+
+// ---------------------------------------------------------------- launch counter
+// Called once per kernel launch by every launcher.
+void count_launch(int n = 1);
+
+// ---------------------------------------------------------------- device status
+// Each translation unit that launches kernels owns a device status word;
+// these read and clear it (after the caller synchronised the stream).
+cudaError_t status_read_clear_generic(int* code);
+cudaError_t status_read_clear_sm100(int* code);
+
+}  // namespace tpla

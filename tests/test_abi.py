@@ -1,0 +1,170 @@
+"""The C-ABI library loads and exports every symbol include/tpla.h declares;
+argument validation rejects bad calls before touching a GPU.  CPU only."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import mla_latent_kv_dim_b200 as tp
+from mla_latent_kv_dim_b200 import _native as N
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "tpla.h")).read()
+    return sorted(set(re.findall(r"TPLA_API\s+[\w\s\*]+?\b(tpla_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("tpla_decode", "tpla_decode_ex", "tpla_decode_workspace_size",
+              "tpla_hadamard_apply", "tpla_vup_combine", "tpla_lse_merge",
+              "tpla_error_string", "tpla_get_device_status", "tpla_version",
+              "tpla_last_cuda_error", "tpla_launch_count"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = tp.lib()
+    for n in _declared():
+        assert hasattr(L, n), n
+    assert tp.version() == 100
+
+
+def test_error_strings():
+    assert tp.error_string(0) == "ok"
+    assert "invalid" in tp.error_string(-1)
+    assert tp.error_string(12345) == "unknown status"
+
+
+def _fake(shape, dtype, ptr=0x10000):
+    """Descriptor with a fake (never dereferenced) aligned pointer."""
+    d = N.TplaTensor()
+    d.data = ptr
+    d.dtype = {torch.bfloat16: 1, torch.float32: 2, torch.int32: 3}[dtype]
+    d.ndim = len(shape)
+    st = 1
+    strides = []
+    for s in reversed(shape):
+        strides.append(st)
+        st *= s
+    strides = list(reversed(strides))
+    for i, s in enumerate(shape):
+        d.shape[i] = s
+        d.stride[i] = strides[i]
+    return d
+
+
+def _call(q, kv, seq, pt, G, rope, out, lse, opts=None, scale=0.07):
+    B = ctypes.byref
+    return tp.lib().tpla_decode_ex(B(q), B(kv), B(seq), B(pt) if pt else None, G, rope,
+                                   ctypes.c_float(scale), B(out), B(lse) if lse else None,
+                                   B(opts) if opts else None, None)
+
+
+def _good(B=2, H=16, G=2, shard=None):
+    q = _fake((B, H, 576), torch.bfloat16)
+    kv = _fake((8, 64, 576), torch.bfloat16)
+    seq = _fake((B,), torch.int32)
+    pt = _fake((B, 4), torch.int32)
+    w = 512 if shard is None else 512 // G
+    out = _fake((B, H, w), torch.float32)
+    lse = _fake((B, H, G if shard is None else 1), torch.float32)
+    return q, kv, seq, pt, out, lse
+
+
+@pytest.mark.parametrize("mutate", [
+    "G3", "G16", "rope2", "q_width", "q_dtype", "kv_page64", "seq_len", "out_width",
+    "lse_width", "nan_scale", "q_misaligned", "q_stride", "shard_range", "reserved",
+])
+def test_validation_rejects_without_launch(mutate):
+    q, kv, seq, pt, out, lse = _good()
+    G, rope, scale, opts = 2, 0, 0.07, None
+    if mutate == "G3":
+        G = 3
+    elif mutate == "G16":
+        G = 16
+    elif mutate == "rope2":
+        rope = 2
+    elif mutate == "q_width":
+        q.shape[2] = 512
+    elif mutate == "q_dtype":
+        q.dtype = 2
+    elif mutate == "kv_page64":
+        kv.shape[1] = 32
+    elif mutate == "seq_len":
+        seq.shape[0] = 3
+    elif mutate == "out_width":
+        out.shape[2] = 256
+    elif mutate == "lse_width":
+        lse.shape[2] = 1
+    elif mutate == "nan_scale":
+        scale = float("nan")
+    elif mutate == "q_misaligned":
+        q.data = 0x10002
+    elif mutate == "q_stride":
+        q.stride[1] = 577
+    elif mutate == "shard_range":
+        opts = N._opts(0, 2, "auto")
+    elif mutate == "reserved":
+        opts = N._opts(0, None, "auto")
+        opts.reserved = 1
+    rc = _call(q, kv, seq, pt, G, rope, out, lse, opts, scale)
+    expect = -2 if mutate == "kv_page64" else -1
+    assert rc == expect, (mutate, rc)
+    assert tp.launch_count() == 0
+
+
+def test_one_shard_shapes_validate():
+    q, kv, seq, pt, out, lse = _good(G=4, shard=1)
+    opts = N._opts(0, 1, "generic")
+    n = ctypes.c_size_t(123)
+    rc = tp.lib().tpla_decode_workspace_size(ctypes.byref(q), ctypes.byref(kv), ctypes.byref(seq),
+                                             ctypes.byref(pt), 4, 1, ctypes.byref(out),
+                                             ctypes.byref(opts), ctypes.byref(n))
+    assert rc == 0
+    # full-width out is rejected in one-shard mode
+    q, kv, seq, pt, out, lse = _good(G=4)
+    rc = tp.lib().tpla_decode_workspace_size(ctypes.byref(q), ctypes.byref(kv), ctypes.byref(seq),
+                                             ctypes.byref(pt), 4, 1, ctypes.byref(out),
+                                             ctypes.byref(opts), ctypes.byref(n))
+    assert rc == -1
+
+
+def test_generic_workspace_size_formula():
+    B, H, G = 3, 16, 2
+    q, kv, seq, pt, out, lse = _good(B=B, H=H, G=G)
+    for splits in (1, 2, 7):
+        opts = N._opts(splits, None, "generic")
+        n = ctypes.c_size_t(0)
+        rc = tp.lib().tpla_decode_workspace_size(ctypes.byref(q), ctypes.byref(kv),
+                                                 ctypes.byref(seq), ctypes.byref(pt), G, 0,
+                                                 ctypes.byref(out), ctypes.byref(opts),
+                                                 ctypes.byref(n))
+        assert rc == 0
+        if splits == 1:
+            assert n.value == 0
+        else:
+            o = splits * B * H * 512 * 4
+            assert n.value == (o + 255) // 256 * 256 + splits * B * H * G * 4
+
+
+def test_hadamard_and_vup_validation():
+    L = tp.lib()
+    buf = _fake((4, 576), torch.bfloat16)
+    assert L.tpla_hadamard_apply(ctypes.byref(buf), 100, None) == -2
+    assert L.tpla_hadamard_apply(ctypes.byref(buf), 2048, None) == -2
+    small = _fake((4, 256), torch.bfloat16)
+    assert L.tpla_hadamard_apply(ctypes.byref(small), 512, None) == -1
+    o = _fake((2, 4, 512), torch.float32)
+    W = _fake((4, 512, 100), torch.bfloat16)
+    y = _fake((2, 4, 100), torch.float32)
+    assert L.tpla_vup_combine(ctypes.byref(o), ctypes.byref(W), ctypes.byref(y), None) == -2
+    W = _fake((3, 512, 128), torch.bfloat16)
+    y = _fake((2, 4, 128), torch.float32)
+    assert L.tpla_vup_combine(ctypes.byref(o), ctypes.byref(W), ctypes.byref(y), None) == -1
+    assert tp.launch_count() == 0
