@@ -155,6 +155,36 @@ TPLA_API int tpla_decode(const tpla_tensor* q, const tpla_tensor* kv_cache,
                 tpla_tensor* lse, tpla_stream_t stream);
 
 /*
+ * tpla_decode_noalloc -- tpla_decode_ex for callers that cannot allocate
+ * device memory while they decode (a caller whose memory pool or arena owns
+ * the whole GPU, a runtime whose allocator must not be re-entered from the
+ * decode call, code paths where cudaMalloc is not allowed).  The source
+ * pages have no counterpart; this is a library convenience.
+ *
+ * Same arguments and results as tpla_decode_ex with opts = {num_splits,
+ * shard, TPLA_KERNEL_AUTO}; there is no workspace argument.  Split-KV
+ * partial results go to one fixed scratch buffer of
+ * TPLA_NOALLOC_SCRATCH_BYTES bytes that the library reserves in device
+ * memory on every GPU where it is loaded and keeps until the process exits.
+ * This call never calls cudaMalloc, cudaFree or any allocating routine.
+ *   - A problem whose workspace (tpla_decode_workspace_size) exceeds that
+ *     capacity is rejected with TPLA_ERR_WORKSPACE before any launch.
+ *   - The first call on a device looks up the buffer's device address
+ *     (cudaGetSymbolAddress, once per device, with that device current);
+ *     make that first call before capturing a stream.
+ *   - All calls on a device share the one buffer and it keeps the previous
+ *     call's contents (nothing needs clearing: every entry read is written
+ *     earlier in the same call).  Calls whose kernels overlap on the GPU,
+ *     e.g. on two streams without ordering, race on the buffer; order them.
+ */
+#define TPLA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+TPLA_API int tpla_decode_noalloc(const tpla_tensor* q, const tpla_tensor* kv_cache,
+                                 const tpla_tensor* seq_lens, const tpla_tensor* page_table,
+                                 int G, int rope_mode, float scale, tpla_tensor* out,
+                                 tpla_tensor* lse, int num_splits, int shard,
+                                 tpla_stream_t stream);
+
+/*
  * tpla_lse_merge -- exact merge of S partial attention results over disjoint
  * key chunks (the log-sum-exp rule of the sequence-split alternative in the
  * feature request's "Directions under investigation").
