@@ -1,15 +1,920 @@
-// tcgen05 / TMA MLA decode kernel for sm_100a (in progress: not yet enabled).
+// MLA / TPLA latent-KV decode on the 5th-generation tensor cores (sm_100a).
+//
+// What it computes (feature request "Bandwidth-optimal tensor-parallel
+// sharding of MLA", sections "Background / problem" and "Directions under
+// investigation"; TPLA abstract; review of arXiv 2508.15881, key machinery
+// and the skeptic's description of Eq. 6 as an unscaled local softmax):
+// for every request b, head h and shard g,
+//   s_t = scale * (q[I_g] . c_t[I_g] + q[R_g] . c_t[R_g])
+//   out[I_g] = softmax_t(s) c_t[I_g],  lse_g = ln sum_t exp(s_t).
+// All heads share one latent row per token, so per request this is a dense
+// [heads x tokens] GEMM (QK^T) followed by a dense [heads x latent] GEMM (PV).
+//
+// Design (B200):
+//  * A CTA pair (cluster of 2, tcgen05 cta_group::2) owns one stream of
+//    128-token tiles.  MMA M = 128 heads: CTA r holds heads [64r, 64r + 64)
+//    of Q in shared memory and the rows of S, P and O for those heads in its
+//    tensor memory.  QK^T uses N = 128 tokens, one 64-token page per CTA;
+//    PV uses N = 128 latent columns, 64 from each CTA.
+//  * Tiles are staged by TMA (no multicast) into a ring of 8 KB slots, each
+//    one [64 rows][64 bf16] box with the 128-byte swizzle the MMA reads
+//    directly: K-major for QK^T, the same bytes MN-major for PV.  The PV
+//    columns are fetched again (mostly from L2) because the pair splits QK
+//    by tokens and PV by latent columns.
+//  * TMEM per CTA: two S buffers (64 columns each) and O (256 columns).
+//    Softmax warps read S with tcgen05.ld, keep a running max per shard and
+//    rescale O in TMEM only when the max grows by more than 2^8 (so P stays
+//    below 256 and bf16); P goes to shared memory for the PV MMA.
+//  * TPLA shards are independent attention problems sharing the cache rows:
+//    a (tile, shard) "unit" is one QK^T, one softmax and one PV, pipelined
+//    two deep (S and P double-buffered).
+//  * Split-KV: a persistent grid of one pair per two SMs walks a balanced
+//    range of the concatenated (request, tile) sequence; requests cut by a
+//    range boundary leave normalised partials + lse in the workspace and
+//    the merge kernel combines them with the log-sum-exp rule (the exact
+//    sequence-split path of the feature request).  Explicit `num_splits`
+//    cuts every request into equal chunks instead.
+//  * Every wait is bounded (2 s); on timeout the kernel records
+//    TPLA_ERR_DEVICE_TIMEOUT, stops issuing work and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include <mutex>
+
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace tpla {
 namespace {
+
+using namespace ptx;
+
+constexpr int kTileTok = 128;      // tokens per tile (two pages)
+constexpr int kStageBytes = 8192;  // one [64][64] bf16 box
+constexpr int kStages = 14;        // TMA ring depth
+constexpr int kQChunks = 9;        // 576 / 64 column chunks of q
+constexpr int kThreads = 192;      // warps 0-3 softmax, 4 producer, 5 MMA
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;      // S buffers: [0, 64), [64, 128)
+constexpr uint32_t kColO = 128;    // O: [128, 384)
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+constexpr int kOffQ = 0;
+constexpr int kOffP = kOffQ + kQChunks * kStageBytes;
+constexpr int kOffRing = kOffP + 4 * kStageBytes;
+constexpr int kOffBar = kOffRing + kStages * kStageBytes;
+constexpr int kNumBars = 2 * kStages + 8;
+constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr int kOffAbort = kOffTmemSlot + 4;
+constexpr int kOffXbuf = kOffAbort + 12;           // float [2][128]
+constexpr int kOffLbuf = kOffXbuf + 2 * 128 * 4;   // float [128][4]
+constexpr int kSmemUsed = kOffLbuf + 128 * 4 * 4;
+constexpr int kSmemBytes = kSmemUsed + 1024;       // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
+
 __device__ int g_status;
+
+__device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
+
+struct Params {
+  const int* seq_lens;
+  const int* page_table;
+  int64_t pt_sb;
+  int num_blocks;   // paged: physical blocks (block index num_blocks reads as zeros)
+  int cap_tokens;   // tokens one request's cache can hold
+  int paged;
+  int B, H, G, split_rope, shard, nsh, d;
+  float scale_log2;  // softmax scale * log2(e)
+  void* out;
+  int out_bf16;
+  int64_t o_sb, o_sh;
+  float* lse;
+  int64_t l_sb, l_sh;
+  float* part_o;  // [slots, H, W]
+  float* part_l;  // [slots, H, nsh]
+  int W;
+  int mode;  // 0 = balanced persistent ranges, 1 = explicit equal splits
+  int P;     // clusters
+  int S;     // explicit splits
+};
+
+// ---------------------------------------------------------------- schedule
+
+__device__ __forceinline__ int req_len(const Params& p, int b) {
+  int L = p.seq_lens[b];
+  if (L < 0 || L > p.cap_tokens) {
+    set_status(TPLA_ERR_DEVICE_BOUNDS);
+    L = L < 0 ? 0 : p.cap_tokens;
+  }
+  return L;
 }
 
-bool sm100_supported(const DecodeProblem&, int) { return false; }
-size_t sm100_workspace_bytes(const DecodeProblem&, int, int) { return 0; }
-cudaError_t launch_decode_sm100(const DecodeProblem&, int, void*, size_t, cudaStream_t) {
-  return cudaErrorNotSupported;
+__device__ __forceinline__ int req_tiles(const Params& p, int b) {
+  return (req_len(p, b) + kTileTok - 1) / kTileTok;
+}
+
+struct Segment {
+  int b, t_lo, t_hi, L;
+  int complete;
+  int slot;
+};
+
+struct Cursor {
+  int b;
+  long long pre, cur, end;
+  int idx;
+};
+
+__device__ void seg_begin(const Params& p, int cl, Cursor& c) {
+  c.idx = 0;
+  if (p.mode == 0) {
+    long long T = 0;
+    for (int b = 0; b < p.B; ++b) T += req_tiles(p, b);
+    // with fewer tiles than clusters only the first T clusters get work, so
+    // that every cluster in a request's range has written its partial slot
+    const long long P = min((long long)p.P, T);
+    if (cl >= P) {
+      c.cur = c.end = 0;
+    } else {
+      c.cur = (long long)cl * T / P;
+      c.end = (long long)(cl + 1) * T / P;
+    }
+    c.b = 0;
+    c.pre = 0;
+  } else {
+    c.b = cl / p.S;
+    c.pre = c.cur = c.end = 0;
+  }
+}
+
+__device__ bool seg_next(const Params& p, int cl, Cursor& c, Segment& s) {
+  if (p.mode == 0) {
+    if (c.cur >= c.end) return false;
+    while (c.b < p.B && c.pre + req_tiles(p, c.b) <= c.cur) {
+      c.pre += req_tiles(p, c.b);
+      ++c.b;
+    }
+    if (c.b >= p.B) return false;
+    const int nt = req_tiles(p, c.b);
+    s.b = c.b;
+    s.L = req_len(p, c.b);
+    s.t_lo = (int)(c.cur - c.pre);
+    s.t_hi = (int)min((long long)nt, c.end - c.pre);
+    s.complete = (s.t_lo == 0 && s.t_hi == nt);
+    s.slot = 2 * cl + (c.idx == 0 ? 0 : 1);
+    c.cur = c.pre + s.t_hi;
+    ++c.idx;
+    return true;
+  }
+  if (c.idx > 0) return false;
+  const int b = cl / p.S, sp = cl % p.S;
+  const int nt = req_tiles(p, b);
+  const int chunk = (nt + p.S - 1) / p.S;
+  s.b = b;
+  s.L = req_len(p, b);
+  s.t_lo = min(nt, sp * chunk);
+  s.t_hi = min(nt, (sp + 1) * chunk);
+  s.complete = p.S == 1;
+  s.slot = 2 * cl;
+  ++c.idx;
+  return true;
+}
+
+// Columns of shard g: latent 64-column chunks [g d/64, (g+1) d/64) and the
+// rope chunk (index 8).  K-steps (16 columns) of the rope chunk this shard
+// uses: all four (replicate) or its own slice (split).
+__device__ __forceinline__ int shard_of(const Params& p, int i) { return p.shard < 0 ? i : p.shard; }
+
+__device__ __forceinline__ void rope_steps(const Params& p, int g, int& k0, int& k1) {
+  if (!p.split_rope) {
+    k0 = 0;
+    k1 = 4;
+  } else {
+    const int per = 4 / p.G;  // 16-column steps per shard (G <= 4)
+    k0 = g * per;
+    k1 = k0 + per;
+  }
+}
+
+// ---------------------------------------------------------------- waits
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 127) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kTimeoutNs) {
+        set_status(TPLA_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+struct Bars {
+  uint32_t base;
+  __device__ uint32_t ring_full(int s) const { return base + 8 * s; }
+  __device__ uint32_t ring_empty(int s) const { return base + 8 * (kStages + s); }
+  __device__ uint32_t q_full() const { return base + 8 * (2 * kStages); }
+  __device__ uint32_t q_empty() const { return base + 8 * (2 * kStages + 1); }
+  __device__ uint32_t s_full(int i) const { return base + 8 * (2 * kStages + 2 + i); }
+  __device__ uint32_t p_full(int i) const { return base + 8 * (2 * kStages + 4 + i); }
+  __device__ uint32_t p_empty(int i) const { return base + 8 * (2 * kStages + 6 + i); }
+};
+
+// ---------------------------------------------------------------- producer
+
+__device__ __forceinline__ int page_block(const Params& p, const Segment& s, int page) {
+  const int npages = (s.L + 63) / 64;
+  if (page >= npages) return p.num_blocks;  // beyond the request: reads as zeros
+  const int blk = p.page_table[(int64_t)s.b * p.pt_sb + page];
+  if (blk < 0 || blk >= p.num_blocks) {
+    set_status(TPLA_ERR_DEVICE_BOUNDS);
+    return p.num_blocks;
+  }
+  return blk;
+}
+
+struct Ring {
+  uint32_t n = 0;  // stages issued / consumed so far
+};
+
+__device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtensorMap* kvmap,
+                         int cl, uint32_t rank, uint32_t sbase, const Bars& bars,
+                         volatile int* abort_flag) {
+  Cursor cur;
+  seg_begin(p, cl, cur);
+  Segment s;
+  uint32_t n = 0, qloads = 0;
+  const uint32_t q_full_c = mapa(bars.q_full(), 0);
+  const int dq = p.d / 64;  // latent chunks per shard
+
+  auto next_slot = [&](uint32_t& slot, uint32_t& full_c) -> bool {
+    slot = n % kStages;
+    if (n >= (uint32_t)kStages) {
+      if (!wait_bar(bars.ring_empty(slot), ((n / kStages) - 1) & 1, abort_flag)) return false;
+    }
+    full_c = mapa(bars.ring_full(slot), 0);
+    if (rank == 0) mbar_arrive_expect_tx(bars.ring_full(slot), 2 * kStageBytes);
+    ++n;
+    return true;
+  };
+  auto load_kv = [&](uint32_t slot, uint32_t full_c, int chunk, int t, int half) {
+    const uint32_t dst = sbase + kOffRing + slot * kStageBytes;
+    if (p.paged) {
+      tma_load_3d_pair(dst, kvmap, 64 * chunk, 0, page_block(p, s, 2 * t + half), full_c);
+    } else {
+      tma_load_3d_pair(dst, kvmap, 64 * chunk, kTileTok * t + 64 * half, s.b, full_c);
+    }
+  };
+
+  while (seg_next(p, cl, cur, s)) {
+    const int nunits = (s.t_hi - s.t_lo) * p.nsh;
+    if (nunits == 0) continue;
+    if (qloads > 0 && !wait_bar(bars.q_empty(), (qloads - 1) & 1, abort_flag)) return;
+    const int nq = p.shard < 0 ? kQChunks : dq + 1;
+    if (rank == 0) mbar_arrive_expect_tx(bars.q_full(), 2 * nq * kStageBytes);
+    for (int i = 0; i < nq; ++i) {
+      const int c = p.shard < 0 ? i : (i < dq ? p.shard * dq + i : 8);
+      tma_load_3d_pair(sbase + kOffQ + c * kStageBytes, qmap, 64 * c, 64 * (int)rank, s.b,
+                       q_full_c);
+    }
+    ++qloads;
+    for (int j = 0; j <= nunits; ++j) {
+      if (j < nunits) {  // QK^T stages of unit j: this CTA's page, shard columns
+        const int t = s.t_lo + j / p.nsh;
+        const int g = shard_of(p, j % p.nsh);
+        for (int i = 0; i <= dq; ++i) {
+          const int c = i < dq ? g * dq + i : 8;
+          uint32_t slot, full_c;
+          if (!next_slot(slot, full_c)) return;
+          load_kv(slot, full_c, c, t, (int)rank);
+        }
+      }
+      if (j >= 1) {  // PV stages of unit j-1: both pages, this CTA's latent half
+        const int k = j - 1;
+        const int t = s.t_lo + k / p.nsh;
+        const int g = shard_of(p, k % p.nsh);
+        for (int nl = 0; nl < p.d / 128; ++nl) {
+          const int ng = g * (p.d / 128) + nl;
+          for (int half = 0; half < 2; ++half) {
+            uint32_t slot, full_c;
+            if (!next_slot(slot, full_c)) return;
+            load_kv(slot, full_c, 2 * ng + (int)rank, t, half);
+          }
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- MMA issuer
+
+__device__ void mma_issuer(const Params& p, int cl, uint32_t sbase, uint32_t tmem,
+                           const Bars& bars, volatile int* abort_flag) {
+  Cursor cur;
+  seg_begin(p, cl, cur);
+  Segment s;
+  uint32_t n = 0, qloads = 0, U0 = 0;
+  const int dq = p.d / 64;
+  const int ng0 = p.shard < 0 ? 0 : p.shard * (p.d / 128);
+
+  auto take = [&](uint32_t& slot) -> bool {
+    slot = n % kStages;
+    if (!wait_bar(bars.ring_full(slot), (n / kStages) & 1, abort_flag)) return false;
+    tc_fence_after();
+    ++n;
+    return true;
+  };
+
+  while (seg_next(p, cl, cur, s)) {
+    const int nunits = (s.t_hi - s.t_lo) * p.nsh;
+    if (nunits == 0) continue;
+    if (!wait_bar(bars.q_full(), qloads & 1, abort_flag)) return;
+    tc_fence_after();
+    ++qloads;
+    for (int j = 0; j <= nunits; ++j) {
+      if (j < nunits) {
+        const uint32_t Ug = U0 + j;
+        const int g = shard_of(p, j % p.nsh);
+        const uint32_t dS = tmem + kColS + 64 * (Ug & 1);
+        uint32_t acc = 0;
+        for (int i = 0; i <= dq; ++i) {
+          const int c = i < dq ? g * dq + i : 8;
+          int k0 = 0, k1 = 4;
+          if (i == dq) rope_steps(p, g, k0, k1);
+          uint32_t slot;
+          if (!take(slot)) return;
+          const uint32_t a0 = sbase + kOffQ + c * kStageBytes;
+          const uint32_t b0 = sbase + kOffRing + slot * kStageBytes;
+          for (int kk = k0; kk < k1; ++kk) {
+            mma_pair_f16(dS, sw128_desc(a0 + 32 * kk, 16, 1024), sw128_desc(b0 + 32 * kk, 16, 1024),
+                         kIdescQK, acc);
+            acc = 1;
+          }
+          mma_commit_pair(bars.ring_empty(slot), 0x3);
+        }
+        mma_commit_pair(bars.s_full(Ug & 1), 0x3);
+        if (j == nunits - 1) mma_commit_pair(bars.q_empty(), 0x3);
+      }
+      if (j >= 1) {
+        const int k = j - 1;
+        const uint32_t Ug = U0 + k;
+        const int g = shard_of(p, k % p.nsh);
+        const bool first = k < p.nsh;  // first tile of this shard in the segment
+        if (!wait_bar(bars.p_full(Ug & 1), (Ug >> 1) & 1, abort_flag)) return;
+        tc_fence_after();
+        const uint32_t pbase = sbase + kOffP + (Ug & 1) * 2 * kStageBytes;
+        for (int nl = 0; nl < p.d / 128; ++nl) {
+          const int ng = g * (p.d / 128) + nl;
+          const uint32_t dO = tmem + kColO + 64 * (ng - ng0);
+          for (int half = 0; half < 2; ++half) {
+            uint32_t slot;
+            if (!take(slot)) return;
+            const uint32_t a0 = pbase + half * kStageBytes;
+            const uint32_t b0 = sbase + kOffRing + slot * kStageBytes;
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (first && half == 0 && kk == 0) ? 0u : 1u;
+              mma_pair_f16(dO, sw128_desc(a0 + 32 * kk, 16, 1024),
+                           sw128_desc(b0 + 2048 * kk, kStageBytes, 1024), kIdescPV, acc);
+            }
+            mma_commit_pair(bars.ring_empty(slot), 0x3);
+          }
+        }
+        mma_commit_pair(bars.p_empty(Ug & 1), 0x3);
+      }
+    }
+    U0 += nunits;
+  }
+}
+
+// ---------------------------------------------------------------- softmax + epilogue
+
+__device__ __forceinline__ void write_out_row(const Params& p, const Segment& s, int head,
+                                              int col0, const float* v, float inv) {
+  if (head >= p.H) return;
+  if (s.complete) {
+    const int64_t off = (int64_t)s.b * p.o_sb + (int64_t)head * p.o_sh + col0;
+    if (p.out_bf16) {
+      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + off;
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        uint4 w;
+        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h2[e] = __floats2bfloat162_rn(v[j + 2 * e] * inv, v[j + 2 * e + 1] * inv);
+        *reinterpret_cast<uint4*>(o + j) = w;
+      }
+    } else {
+      float* o = reinterpret_cast<float*>(p.out) + off;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4*>(o + j) =
+            make_float4(v[j] * inv, v[j + 1] * inv, v[j + 2] * inv, v[j + 3] * inv);
+    }
+  } else {
+    float* o = p.part_o + ((int64_t)s.slot * p.H + head) * p.W + col0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4)
+      *reinterpret_cast<float4*>(o + j) =
+          make_float4(v[j] * inv, v[j + 1] * inv, v[j + 2] * inv, v[j + 3] * inv);
+  }
+}
+
+__device__ __forceinline__ void write_lse(const Params& p, const Segment& s, int head, int i,
+                                          float v) {
+  if (head >= p.H) return;
+  if (s.complete) {
+    if (p.lse) p.lse[(int64_t)s.b * p.l_sb + (int64_t)head * p.l_sh + i] = v;
+  } else {
+    p.part_l[((int64_t)s.slot * p.H + head) * p.nsh + i] = v;
+  }
+}
+
+__device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t sbase,
+                              uint8_t* smem, uint32_t tmem, const Bars& bars,
+                              volatile int* abort_flag) {
+  const int tid = threadIdx.x;  // 0..127 = TMEM lane
+  const int warp = tid >> 5;
+  const int half = tid >> 6, hl = tid & 63;
+  const int head = 64 * (int)rank + hl;
+  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  float* xbuf = reinterpret_cast<float*>(smem + kOffXbuf);
+  float* lbuf = reinterpret_cast<float*>(smem + kOffLbuf);
+  const uint32_t pf_c[2] = {mapa(bars.p_full(0), 0), mapa(bars.p_full(1), 0)};
+  const int ng0 = p.shard < 0 ? 0 : p.shard * (p.d / 128);
+  const int nchunks = p.d / 128;
+
+  Cursor cur;
+  seg_begin(p, cl, cur);
+  Segment s;
+  uint32_t U = 0;
+  while (seg_next(p, cl, cur, s)) {
+    const int nunits = (s.t_hi - s.t_lo) * p.nsh;
+    if (nunits == 0) {  // empty chunk: out 0, lse -inf
+      float z[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) z[j] = 0.f;
+      for (int i = 0; i < p.nsh; ++i) {
+        const int g = shard_of(p, i);
+        for (int nl = 0; nl < nchunks; ++nl) {
+          const int ng = g * nchunks + nl;
+          const int col = (p.shard < 0 ? 128 * ng : 128 * nl) + 64 * half;
+          write_out_row(p, s, head, col, z, 0.f);
+          write_out_row(p, s, head, col + 32, z, 0.f);
+        }
+        if (half == 0) write_lse(p, s, head, i, -INFINITY);
+      }
+      continue;
+    }
+    float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    float l[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k = 0; k < nunits; ++k) {
+      const uint32_t Ug = U + k;
+      const int i = k % p.nsh;
+      const int g = shard_of(p, i);
+      const int t = s.t_lo + k / p.nsh;
+      if (!wait_bar(bars.s_full(Ug & 1), (Ug >> 1) & 1, abort_flag)) return;
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tmem + lane_base + kColS + 64 * (Ug & 1), r0);
+      tmem_ld32(tmem + lane_base + kColS + 64 * (Ug & 1) + 32, r1);
+      tmem_wait_ld();
+      const int nv = max(0, min(64, s.L - (kTileTok * t + 64 * half)));
+      float x[64];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        x[j] = j < nv ? __uint_as_float(r0[j]) * p.scale_log2 : -INFINITY;
+        x[j + 32] = j + 32 < nv ? __uint_as_float(r1[j]) * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, fmaxf(x[j], x[j + 32]));
+      }
+      xbuf[(Ug & 1) * 128 + tid] = mx;
+      named_bar_sync(1, 128);
+      mx = fmaxf(mx, xbuf[(Ug & 1) * 128 + (tid ^ 64)]);
+      float mi = m[i];
+      float factor = 1.f;
+      int resc = 0;
+      if (mi == -INFINITY) {
+        mi = mx;
+      } else if (mx > mi + kRescaleThreshold) {
+        factor = ex2(mi - mx);
+        mi = mx;
+        resc = 1;
+      }
+      m[i] = mi;
+      l[i] *= factor;
+      if (__any_sync(0xffffffffu, resc)) {
+        // O of this shard was last written by an earlier PV: wait for all
+        // issued PVs (up to unit Ug - 1), then rescale in TMEM
+        if (!wait_bar(bars.p_empty((Ug - 1) & 1), ((Ug - 1) >> 1) & 1, abort_flag)) return;
+        tc_fence_after();
+        for (int nl = 0; nl < nchunks; ++nl) {
+          const int ng = g * nchunks + nl;
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const uint32_t ta = tmem + lane_base + kColO + 64 * (ng - ng0) + 32 * c2;
+            uint32_t o[32];
+            tmem_ld32(ta, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * factor);
+            tmem_st32(ta, o);
+          }
+        }
+        tmem_wait_st();
+      }
+      // P = 2^(x - m) in bf16 (masked tokens give 0); l sums the rounded values
+      uint32_t pk[32];
+      float lsum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(ex2(x[2 * j] - mi), ex2(x[2 * j + 1] - mi));
+        float2 f2 = __bfloat1622float2(h2);
+        lsum += f2.x + f2.y;
+        pk[j] = *reinterpret_cast<uint32_t*>(&h2);
+      }
+      l[i] += lsum;
+      if (Ug >= 2) {
+        if (!wait_bar(bars.p_empty(Ug & 1), ((Ug - 2) >> 1) & 1, abort_flag)) return;
+      }
+      const uint32_t prow = sbase + kOffP + (Ug & 1) * 2 * kStageBytes + half * kStageBytes + hl * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(prow + ((c ^ (hl & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive_cluster(pf_c[Ug & 1]);
+    }
+    U += nunits;
+    // epilogue: all PVs of the segment done
+    if (!wait_bar(bars.p_empty((U - 1) & 1), ((U - 1) >> 1) & 1, abort_flag)) return;
+    tc_fence_after();
+    for (int i = 0; i < p.nsh; ++i) lbuf[tid * 4 + i] = l[i];
+    named_bar_sync(1, 128);
+    for (int i = 0; i < p.nsh; ++i) {
+      const int g = shard_of(p, i);
+      const float lt = l[i] + lbuf[(tid ^ 64) * 4 + i];
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float lse = lt > 0.f ? (m[i] + log2f(lt)) * kLn2 : -INFINITY;
+      for (int nl = 0; nl < nchunks; ++nl) {
+        const int ng = g * nchunks + nl;
+        const int col = (p.shard < 0 ? 128 * ng : 128 * nl) + 64 * half;
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + kColO + 64 * (ng - ng0) + 32 * c2, o);
+          tmem_wait_ld();
+          write_out_row(p, s, head, col + 32 * c2, reinterpret_cast<const float*>(o), inv);
+        }
+      }
+      if (half == 0) write_lse(p, s, head, i, lse);
+    }
+    tc_fence_before();
+    named_bar_sync(1, 128);
+  }
+}
+
+// ---------------------------------------------------------------- kernel
+
+__global__ void __launch_bounds__(kThreads, 1)
+tpla_decode_sm100_kernel(const __grid_constant__ CUtensorMap qmap,
+                         const __grid_constant__ CUtensorMap kvmap, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cl = (int)cluster_id_x();
+  Bars bars{sbase + kOffBar};
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bars.ring_full(s), 1);
+      mbar_init(bars.ring_empty(s), 1);
+    }
+    mbar_init(bars.q_full(), 1);
+    mbar_init(bars.q_empty(), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars.s_full(i), 1);
+      mbar_init(bars.p_full(i), 8);  // 4 softmax warps x 2 CTAs
+      mbar_init(bars.p_empty(i), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch(&qmap);
+    tma_prefetch(&kvmap);
+  }
+  if (warp == 5) {
+    tmem_alloc_pair(sbase + kOffTmemSlot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemSlot);
+
+  if (warp == 4) {
+    if (lane == 0) producer(p, &qmap, &kvmap, cl, rank, sbase, bars, abort_flag);
+  } else if (warp == 5) {
+    if (lane == 0 && rank == 0) mma_issuer(p, cl, sbase, tmem, bars, abort_flag);
+  } else {
+    softmax_warps(p, cl, rank, sbase, smem, tmem, bars, abort_flag);
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- merge of partial slots
+
+constexpr int kMergeThreads = 128;
+
+__global__ void __launch_bounds__(kMergeThreads)
+sm100_merge_kernel(const Params p) {
+  const int b = blockIdx.x / p.H;
+  const int h = blockIdx.x % p.H;
+  __shared__ long long red[2][kMergeThreads];
+  long long pre = 0, tot = 0;
+  for (int bb = threadIdx.x; bb < p.B; bb += kMergeThreads) {
+    const long long nt = req_tiles(p, bb);
+    tot += nt;
+    if (bb < b) pre += nt;
+  }
+  red[0][threadIdx.x] = pre;
+  red[1][threadIdx.x] = tot;
+  __syncthreads();
+  for (int o = kMergeThreads / 2; o; o >>= 1) {
+    if (threadIdx.x < o) {
+      red[0][threadIdx.x] += red[0][threadIdx.x + o];
+      red[1][threadIdx.x] += red[1][threadIdx.x + o];
+    }
+    __syncthreads();
+  }
+  pre = red[0][0];
+  const long long T = red[1][0];
+  const int nt = req_tiles(p, b);
+  const int cw = p.W / p.nsh;
+
+  auto write_final = [&](int k, int col, float v) {
+    const int64_t off = (int64_t)b * p.o_sb + (int64_t)h * p.o_sh + k * cw + col;
+    if (p.out_bf16)
+      reinterpret_cast<__nv_bfloat16*>(p.out)[off] = __float2bfloat16_rn(v);
+    else
+      reinterpret_cast<float*>(p.out)[off] = v;
+  };
+
+  if (nt == 0) {  // empty request
+    for (int k = 0; k < p.nsh; ++k) {
+      for (int c = threadIdx.x; c < cw; c += kMergeThreads) write_final(k, c, 0.f);
+      if (p.lse && threadIdx.x == 0) p.lse[(int64_t)b * p.l_sb + (int64_t)h * p.l_sh + k] = -INFINITY;
+    }
+    return;
+  }
+  int s_lo, s_hi;  // cluster range
+  const long long P = min((long long)p.P, T);  // clusters that received work
+  if (p.mode == 0) {
+    s_lo = (int)(((pre + 1) * P + T - 1) / T - 1);
+    s_hi = (int)(((pre + nt) * P + T - 1) / T - 1);
+    if (s_lo == s_hi) return;  // one cluster wrote the final result
+  } else {
+    if (p.S == 1) return;
+    s_lo = b * p.S;
+    s_hi = b * p.S + p.S - 1;
+  }
+  auto slot_of = [&](int c) -> int {
+    if (p.mode == 0) {
+      const long long start = (long long)c * T / P;
+      return (c == s_lo && start < pre) ? 2 * c + 1 : 2 * c;
+    }
+    return 2 * c;
+  };
+  for (int k = 0; k < p.nsh; ++k) {
+    float M = -INFINITY;
+    for (int c = s_lo; c <= s_hi; ++c)
+      M = fmaxf(M, p.part_l[((int64_t)slot_of(c) * p.H + h) * p.nsh + k]);
+    float z = 0.f;
+    if (M != -INFINITY)
+      for (int c = s_lo; c <= s_hi; ++c) {
+        const float ls = p.part_l[((int64_t)slot_of(c) * p.H + h) * p.nsh + k];
+        if (ls != -INFINITY) z += expf(ls - M);
+      }
+    const float total = M == -INFINITY ? -INFINITY : M + logf(z);
+    for (int col = threadIdx.x; col < cw; col += kMergeThreads) {
+      float acc = 0.f;
+      if (total != -INFINITY)
+        for (int c = s_lo; c <= s_hi; ++c) {
+          const int sl = slot_of(c);
+          const float ls = p.part_l[((int64_t)sl * p.H + h) * p.nsh + k];
+          if (ls == -INFINITY) continue;
+          acc = fmaf(expf(ls - total), p.part_o[((int64_t)sl * p.H + h) * p.W + k * cw + col], acc);
+        }
+      write_final(k, col, acc);
+    }
+    if (p.lse && threadIdx.x == 0) p.lse[(int64_t)b * p.l_sb + (int64_t)h * p.l_sh + k] = total;
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+struct DeviceInfo {
+  bool init = false;
+  bool sm100 = false;
+  int max_clusters = 0;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+cudaError_t launch_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int clusters,
+                          cudaStream_t stream) {
+  cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaSuccess;
+}
+
+const DeviceInfo& device_info(int dev) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev & 63];
+  if (d.init) return d;
+  d.init = true;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return d;
+  }
+  if (major != 10 || minor != 0) return d;
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn) {
+      cudaGetLastError();
+      return d;
+    }
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  if (cudaFuncSetAttribute(tpla_decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemBytes) != cudaSuccess) {
+    cudaGetLastError();
+    return d;
+  }
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  launch_config(cfg, attr, sms / 2, nullptr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, tpla_decode_sm100_kernel, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return d;
+  }
+  d.max_clusters = n;
+  d.sm100 = true;
+  return d;
+}
+
+bool encode_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                uint64_t stride1_bytes, uint64_t stride2_bytes) {
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_slots(const DecodeProblem& p, int num_splits, int max_clusters) {
+  if (num_splits == 0) return 2 * max_clusters;
+  if (num_splits == 1) return 0;
+  return 2 * p.B * num_splits;
+}
+
+}  // namespace
+
+bool sm100_supported(const DecodeProblem& p, int device) {
+  if (device < 0 || device >= 64) return false;
+  if (!(p.G == 1 || p.G == 2 || p.G == 4)) return false;
+  if (p.H < 1 || p.H > 128) return false;
+  if (p.cache_rows > (1 << 30) || (p.page_table && p.num_blocks >= (1LL << 31) - 1)) return false;
+  if (p.page_table && p.max_pages > (1 << 24)) return false;
+  // 16-byte vector stores of out rows
+  const int vec = p.out_bf16 ? 8 : 4;
+  if ((reinterpret_cast<uintptr_t>(p.out) & 15u) || (p.o_sb % vec) || (p.o_sh % vec)) return false;
+  const DeviceInfo& d = device_info(device);
+  return d.sm100;
+}
+
+size_t sm100_workspace_bytes(const DecodeProblem& p, int num_splits, int device) {
+  const DeviceInfo& d = device_info(device);
+  const int slots = num_slots(p, num_splits, d.max_clusters);
+  if (slots == 0) return 0;
+  const size_t o = (size_t)slots * p.H * p.out_width * sizeof(float);
+  return ((o + 255) / 256) * 256 + (size_t)slots * p.H * p.n_shards * sizeof(float);
+}
+
+cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* ws, size_t ws_bytes,
+                                cudaStream_t stream) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const DeviceInfo& d = device_info(dev);
+  if (!d.sm100) return cudaErrorNotSupported;
+  CUtensorMap qmap, kvmap;
+  if (!encode_map(&qmap, dp.q, kWidth, dp.H, dp.B, dp.q_sh * 2, dp.q_sb * 2))
+    return cudaErrorInvalidValue;
+  if (dp.page_table) {
+    if (!encode_map(&kvmap, dp.cache, kWidth, kBlock, dp.num_blocks, dp.c_s1 * 2, dp.c_s0 * 2))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!encode_map(&kvmap, dp.cache, kWidth, dp.cache_rows, dp.B, dp.c_s1 * 2, dp.c_s0 * 2))
+      return cudaErrorInvalidValue;
+  }
+  Params p{};
+  p.seq_lens = dp.seq_lens;
+  p.page_table = dp.page_table;
+  p.pt_sb = dp.pt_sb;
+  p.num_blocks = (int)dp.num_blocks;
+  p.cap_tokens = (int)dp.cache_rows;
+  p.paged = dp.page_table != nullptr;
+  p.B = dp.B;
+  p.H = dp.H;
+  p.G = dp.G;
+  p.split_rope = dp.rope_mode == TPLA_ROPE_SPLIT;
+  p.shard = dp.shard;
+  p.nsh = dp.n_shards;
+  p.d = kLatent / dp.G;
+  p.scale_log2 = (float)((double)dp.scale * 1.4426950408889634);
+  p.out = dp.out;
+  p.out_bf16 = dp.out_bf16;
+  p.o_sb = dp.o_sb;
+  p.o_sh = dp.o_sh;
+  p.lse = dp.lse;
+  p.l_sb = dp.l_sb;
+  p.l_sh = dp.l_sh;
+  p.W = dp.out_width;
+  const int slots = num_slots(dp, num_splits, d.max_clusters);
+  if (slots > 0) {
+    const size_t o = (size_t)slots * dp.H * dp.out_width * sizeof(float);
+    const size_t need = ((o + 255) / 256) * 256 + (size_t)slots * dp.H * dp.n_shards * sizeof(float);
+    if (!ws || ws_bytes < need) return cudaErrorInvalidValue;
+    p.part_o = reinterpret_cast<float*>(ws);
+    p.part_l = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + ((o + 255) / 256) * 256);
+  }
+  int clusters;
+  if (num_splits == 0) {
+    p.mode = 0;
+    p.P = d.max_clusters;
+    p.S = 1;
+    clusters = d.max_clusters;
+  } else {
+    p.mode = 1;
+    p.S = num_splits;
+    p.P = dp.B * num_splits;
+    clusters = p.P;
+  }
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  launch_config(cfg, attr, clusters, stream);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tpla_decode_sm100_kernel, qmap, kvmap, p);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  if (p.mode == 0 || p.S > 1) {
+    sm100_merge_kernel<<<dp.B * dp.H, kMergeThreads, 0, stream>>>(p);
+    count_launch();
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 cudaError_t status_read_clear_sm100(int* code) {
@@ -23,4 +928,5 @@ cudaError_t status_read_clear_sm100(int* code) {
   *code = v;
   return e;
 }
+
 }  // namespace tpla

@@ -95,6 +95,9 @@ def test_bf16_output(cuda_dev, kernel):
     w = make_inputs(2, 128, [513, 64], paged=True, decay=True, seed=51)
     out, lse = run(cuda_dev, w, 2, "replicate", kernel, out_dtype=torch.bfloat16)
     ro, rl = oracle_decode(w, 2, "replicate")
+    # a bf16 output stores the result in bf16: compare with the oracle's
+    # result rounded the same way (round-to-nearest-even)
+    ro = to_np(torch.from_numpy(ro).to(torch.bfloat16))
     assert_out_close(out, ro)
     assert_lse_close(lse, rl)
 
