@@ -56,6 +56,10 @@ def parse_args():
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-extras", action="store_true", help="skip the per-G sweep")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="fewer requests of the same shape (profiling captures)")
+    ap.add_argument("--profile", action="store_true",
+                    help="decode launches only: warmup + steps, one short JSON line")
     return ap.parse_args()
 
 
@@ -459,8 +463,43 @@ def _sm100_used(tp, q, cache, seq, pt, G, rope, out, args):
         return False
 
 
+def run_profile(args):
+    """Decode launches only (for ncu captures): W warm-up + K timed launches."""
+    import mla_latent_kv_dim_b200 as tp
+    dev = torch.device("cuda", 0)
+    w = make_workload(args.config, batch=args.batch)
+    q, cache, seq = w.q.to(dev), w.cache.to(dev), w.seq_lens.to(dev)
+    pt = None if w.page_table is None else w.page_table.to(dev)
+    out = torch.empty((w.B, w.H, LATENT), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.B, w.H, args.G), dtype=torch.float32, device=dev)
+    need = tp.decode_workspace_size(q, cache, seq, pt, args.G, args.rope, out,
+                                    num_splits=args.num_splits, kernel=args.kernel)
+    ws = torch.empty(max(16, need), dtype=torch.uint8, device=dev)
+
+    def once():
+        tp.decode(q, cache, seq, pt, args.G, args.rope, w.scale, out=out, lse=lse,
+                  num_splits=args.num_splits, kernel=args.kernel, workspace=ws)
+
+    for _ in range(args.warmup):
+        once()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        once()
+    b.record()
+    torch.cuda.synchronize()
+    t = a.elapsed_time(b) / 1e3 / args.steps
+    nb = w.latent_kv_bytes(args.G)
+    print(json.dumps({"profile": args.config, "B": w.B, "G": args.G, "decode_us": round(t * 1e6, 1),
+                      "GB_s": round(nb / t / 1e9, 1), "status": tp.device_status()}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.profile:
+        return run_profile(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -34,7 +34,7 @@
 //    the merge kernel combines them with the log-sum-exp rule (the exact
 //    sequence-split path of the feature request).  Explicit `num_splits`
 //    cuts every request into equal chunks instead.
-//  * Every wait is bounded (2 s); on timeout the kernel records
+//  * Every wait is bounded (about 2 s); on timeout the kernel records
 //    TPLA_ERR_DEVICE_TIMEOUT, stops issuing work and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -54,13 +54,17 @@ using namespace ptx;
 
 constexpr int kTileTok = 128;      // tokens per tile (two pages)
 constexpr int kStageBytes = 8192;  // one [64][64] bf16 box
-constexpr int kStages = 14;        // TMA ring depth
+constexpr int kProducers = 4;      // TMA-issuing warps
+constexpr int kStages = 12;        // TMA ring depth (a multiple of kProducers)
 constexpr int kQChunks = 9;        // 576 / 64 column chunks of q
-constexpr int kThreads = 192;      // warps 0-3 softmax, 4 producer, 5 MMA
+constexpr int kWarpProducer0 = 4;  // warps 0-3 softmax, 4-7 producers, 8-11 MMA issuers
+constexpr int kWarpIssuer0 = kWarpProducer0 + kProducers;
+constexpr int kThreads = 32 * (kWarpIssuer0 + 4);
+static_assert(kStages % kProducers == 0, "each ring slot belongs to one producer");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // S buffers: [0, 64), [64, 128)
 constexpr uint32_t kColO = 128;    // O: [128, 384)
-constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s at full clock
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -68,7 +72,7 @@ constexpr int kOffQ = 0;
 constexpr int kOffP = kOffQ + kQChunks * kStageBytes;
 constexpr int kOffRing = kOffP + 4 * kStageBytes;
 constexpr int kOffBar = kOffRing + kStages * kStageBytes;
-constexpr int kNumBars = 2 * kStages + 8;
+constexpr int kNumBars = 5 * kStages + 8;  // full[4][kStages], empty[kStages], 8 more
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemSlot + 4;
 constexpr int kOffXbuf = kOffAbort + 12;           // float [2][128]
@@ -206,14 +210,17 @@ __device__ __forceinline__ void rope_steps(const Params& p, int g, int& k0, int&
 
 // ---------------------------------------------------------------- waits
 
+// Bounded wait.  The bound uses the SM cycle counter: reading %globaltimer
+// costs about half a microsecond, which would throttle every pipeline
+// hand-off that has to wait.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 127) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kTimeoutNs) {
+      if (clock64() - t0 > kTimeoutCycles) {
         set_status(TPLA_ERR_DEVICE_TIMEOUT);
         *abort_flag = 1;
         return false;
@@ -222,59 +229,105 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// Warp-uniform variant: lane 0 polls, the result is broadcast.
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity,
+                                              volatile int* abort_flag) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag);
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Ring "full" barriers exist per (slot, consuming issuer).  A barrier phase
+// wait only tells phases apart by parity, so a waiter must never be two
+// phases away from the barrier; one shared full barrier per slot breaks that
+// when an issuer skips the other issuers' stages and runs ahead.  With one
+// full barrier per (slot, issuer) every barrier has a single consumer that
+// takes its phases strictly in order.
 struct Bars {
   uint32_t base;
-  __device__ uint32_t ring_full(int s) const { return base + 8 * s; }
-  __device__ uint32_t ring_empty(int s) const { return base + 8 * (kStages + s); }
-  __device__ uint32_t q_full() const { return base + 8 * (2 * kStages); }
-  __device__ uint32_t q_empty() const { return base + 8 * (2 * kStages + 1); }
-  __device__ uint32_t s_full(int i) const { return base + 8 * (2 * kStages + 2 + i); }
-  __device__ uint32_t p_full(int i) const { return base + 8 * (2 * kStages + 4 + i); }
-  __device__ uint32_t p_empty(int i) const { return base + 8 * (2 * kStages + 6 + i); }
+  __device__ uint32_t ring_full(int s, int owner) const { return base + 8 * (owner * kStages + s); }
+  __device__ uint32_t ring_empty(int s) const { return base + 8 * (4 * kStages + s); }
+  __device__ uint32_t q_full() const { return base + 8 * (5 * kStages); }
+  __device__ uint32_t q_empty() const { return base + 8 * (5 * kStages + 1); }
+  __device__ uint32_t s_full(int i) const { return base + 8 * (5 * kStages + 2 + i); }
+  __device__ uint32_t p_full(int i) const { return base + 8 * (5 * kStages + 4 + i); }
+  __device__ uint32_t p_empty(int i) const { return base + 8 * (5 * kStages + 6 + i); }
 };
 
 // ---------------------------------------------------------------- producer
 
-__device__ __forceinline__ int page_block(const Params& p, const Segment& s, int page) {
-  const int npages = (s.L + 63) / 64;
-  if (page >= npages) return p.num_blocks;  // beyond the request: reads as zeros
-  const int blk = p.page_table[(int64_t)s.b * p.pt_sb + page];
-  if (blk < 0 || blk >= p.num_blocks) {
-    set_status(TPLA_ERR_DEVICE_BOUNDS);
-    return p.num_blocks;
-  }
-  return blk;
-}
+// Physical block ids of one request, fetched 32 pages at a time by the
+// whole producer warp (one coalesced load) and handed to lane 0 by shuffle,
+// so TMA issue never waits on a page-table load.
+struct PageWindow {
+  int b = -1, base = 0, blk = 0;
 
-struct Ring {
-  uint32_t n = 0;  // stages issued / consumed so far
+  __device__ int get(const Params& p, const Segment& s, int page, int lane) {
+    const int npages = (s.L + 63) / 64;
+    if (page >= npages) return p.num_blocks;  // beyond the request: reads as zeros
+    if (s.b != b || page < base || page >= base + 32) {
+      b = s.b;
+      base = page;
+      const int pg = base + lane;
+      int v = p.num_blocks;
+      if (pg < npages) {
+        v = p.page_table[(int64_t)s.b * p.pt_sb + pg];
+        if (v < 0 || v >= p.num_blocks) {
+          set_status(TPLA_ERR_DEVICE_BOUNDS);
+          v = p.num_blocks;
+        }
+      }
+      blk = v;
+    }
+    return __shfl_sync(0xffffffffu, blk, page - base);
+  }
 };
 
+// Runs on all 32 lanes of the producer warp (uniform control flow); lane 0
+// issues the barrier arrivals and TMA copies.
+//
+// A thread issuing TMA copies waits a few hundred cycles per copy, so one
+// producer cannot feed the pipeline: kProducers warps share the stage
+// sequence, stage n being loaded by warp n % kProducers.  kStages is a
+// multiple of kProducers, so every ring slot (and its empty barrier) always
+// belongs to the same producer, which takes its phases in order.
 __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtensorMap* kvmap,
-                         int cl, uint32_t rank, uint32_t sbase, const Bars& bars,
+                         int cl, int pid, uint32_t rank, uint32_t sbase, const Bars& bars,
                          volatile int* abort_flag) {
+  const int lane = threadIdx.x & 31;
+  const bool leader_lane = lane == 0;
   Cursor cur;
   seg_begin(p, cl, cur);
   Segment s;
-  uint32_t n = 0, qloads = 0;
+  PageWindow win;
+  uint32_t n = 0, qloads = 0, U0 = 0;
   const uint32_t q_full_c = mapa(bars.q_full(), 0);
   const int dq = p.d / 64;  // latent chunks per shard
+  const int hsplit = (p.d / 128 + 1) / 2;  // PV chunks [0, hsplit) -> issuer 2, rest -> 3
 
-  auto next_slot = [&](uint32_t& slot, uint32_t& full_c) -> bool {
-    slot = n % kStages;
-    if (n >= (uint32_t)kStages) {
-      if (!wait_bar(bars.ring_empty(slot), ((n / kStages) - 1) & 1, abort_flag)) return false;
+  // Stage n goes to slot n % kStages once the slot's previous stage was
+  // released, and signals the full barrier of its consuming issuer `owner`.
+  // Returns 1 when this warp loads stage n, 0 when another producer does,
+  // -1 on abort.  Warp-uniform.
+  auto next_slot = [&](uint32_t& slot, uint32_t& full_c, int owner) -> int {
+    const uint32_t me = n++;
+    if (me % kProducers != (uint32_t)pid) return 0;
+    slot = me % kStages;
+    if (me >= (uint32_t)kStages) {
+      if (!wait_bar_warp(bars.ring_empty(slot), ((me / kStages) - 1) & 1, abort_flag))
+        return -1;
     }
-    full_c = mapa(bars.ring_full(slot), 0);
-    if (rank == 0) mbar_arrive_expect_tx(bars.ring_full(slot), 2 * kStageBytes);
-    ++n;
-    return true;
+    full_c = mapa(bars.ring_full(slot, owner), 0);
+    if (rank == 0 && leader_lane)
+      mbar_arrive_expect_tx(bars.ring_full(slot, owner), 2 * kStageBytes);
+    return 1;
   };
   auto load_kv = [&](uint32_t slot, uint32_t full_c, int chunk, int t, int half) {
     const uint32_t dst = sbase + kOffRing + slot * kStageBytes;
     if (p.paged) {
-      tma_load_3d_pair(dst, kvmap, 64 * chunk, 0, page_block(p, s, 2 * t + half), full_c);
-    } else {
+      const int blk = win.get(p, s, 2 * t + half, lane);
+      if (leader_lane) tma_load_3d_pair(dst, kvmap, 64 * chunk, 0, blk, full_c);
+    } else if (leader_lane) {
       tma_load_3d_pair(dst, kvmap, 64 * chunk, kTileTok * t + 64 * half, s.b, full_c);
     }
   };
@@ -282,24 +335,30 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
   while (seg_next(p, cl, cur, s)) {
     const int nunits = (s.t_hi - s.t_lo) * p.nsh;
     if (nunits == 0) continue;
-    if (qloads > 0 && !wait_bar(bars.q_empty(), (qloads - 1) & 1, abort_flag)) return;
-    const int nq = p.shard < 0 ? kQChunks : dq + 1;
-    if (rank == 0) mbar_arrive_expect_tx(bars.q_full(), 2 * nq * kStageBytes);
-    for (int i = 0; i < nq; ++i) {
-      const int c = p.shard < 0 ? i : (i < dq ? p.shard * dq + i : 8);
-      tma_load_3d_pair(sbase + kOffQ + c * kStageBytes, qmap, 64 * c, 64 * (int)rank, s.b,
-                       q_full_c);
+    if (pid == 0) {  // q of this segment, once its previous user is done
+      if (qloads > 0 && !wait_bar_warp(bars.q_empty(), (qloads - 1) & 1, abort_flag)) return;
+      const int nq = p.shard < 0 ? kQChunks : dq + 1;
+      if (leader_lane) {
+        if (rank == 0) mbar_arrive_expect_tx(bars.q_full(), 2 * nq * kStageBytes);
+        for (int i = 0; i < nq; ++i) {
+          const int c = p.shard < 0 ? i : (i < dq ? p.shard * dq + i : 8);
+          tma_load_3d_pair(sbase + kOffQ + c * kStageBytes, qmap, 64 * c, 64 * (int)rank, s.b,
+                           q_full_c);
+        }
+      }
     }
     ++qloads;
     for (int j = 0; j <= nunits; ++j) {
       if (j < nunits) {  // QK^T stages of unit j: this CTA's page, shard columns
         const int t = s.t_lo + j / p.nsh;
         const int g = shard_of(p, j % p.nsh);
+        const int owner = (int)((U0 + j) & 1);
         for (int i = 0; i <= dq; ++i) {
           const int c = i < dq ? g * dq + i : 8;
           uint32_t slot, full_c;
-          if (!next_slot(slot, full_c)) return;
-          load_kv(slot, full_c, c, t, (int)rank);
+          const int r = next_slot(slot, full_c, owner);
+          if (r < 0) return;
+          if (r > 0) load_kv(slot, full_c, c, t, (int)rank);
         }
       }
       if (j >= 1) {  // PV stages of unit j-1: both pages, this CTA's latent half
@@ -310,91 +369,139 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
           const int ng = g * (p.d / 128) + nl;
           for (int half = 0; half < 2; ++half) {
             uint32_t slot, full_c;
-            if (!next_slot(slot, full_c)) return;
-            load_kv(slot, full_c, 2 * ng + (int)rank, t, half);
+            const int r = next_slot(slot, full_c, nl < hsplit ? 2 : 3);
+            if (r < 0) return;
+            if (r > 0) load_kv(slot, full_c, 2 * ng + (int)rank, t, half);
           }
         }
       }
     }
+    U0 += nunits;
   }
 }
 
-// ---------------------------------------------------------------- MMA issuer
+// ---------------------------------------------------------------- MMA issuers
+//
+// One thread issuing tcgen05.mma waits ~150 cycles per instruction whatever
+// its shape, while a 128 x 128 x 16 pair MMA keeps the tensor pipe busy for
+// only 32 cycles per SM.  So four warps of the leader CTA issue MMAs into
+// independent accumulators: role 0/1 = QK^T of even/odd units (S buffer
+// Ug & 1), role 2/3 = PV of the first/second half of the unit's 128-wide
+// latent chunks (disjoint O columns).  Every issuer walks the producer's
+// stage sequence and consumes (waits for, multiplies, releases) only its
+// own ring slots; a commit tracks only the issuing thread's MMAs, so each
+// issuer releases its own slots and signals its own barriers.
 
-__device__ void mma_issuer(const Params& p, int cl, uint32_t sbase, uint32_t tmem,
+__device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, uint32_t tmem,
                            const Bars& bars, volatile int* abort_flag) {
   Cursor cur;
   seg_begin(p, cl, cur);
   Segment s;
   uint32_t n = 0, qloads = 0, U0 = 0;
   const int dq = p.d / 64;
-  const int ng0 = p.shard < 0 ? 0 : p.shard * (p.d / 128);
+  const int nchunks = p.d / 128;
+  const int ng0 = p.shard < 0 ? 0 : p.shard * nchunks;
+  const bool qk = role < 2;
+  const uint32_t parity_role = (uint32_t)(role & 1);
+  // PV roles split the unit's latent chunks: [0, h) and [h, nchunks)
+  const int hsplit = (nchunks + 1) / 2;
+  const int nl_lo = role == 2 ? 0 : hsplit;
+  const int nl_hi = role == 2 ? hsplit : nchunks;
+  // Descriptor templates; an operand at byte offset `o` from a region start
+  // is template + (o >> 4) (shared memory is below 256 KB, so the 14-bit
+  // start-address field never overflows).
+  const uint64_t dQ = sw128_desc(sbase + kOffQ, 16, 1024);               // K-major q
+  const uint64_t dRk = sw128_desc(sbase + kOffRing, 16, 1024);           // K-major ring
+  const uint64_t dRm = sw128_desc(sbase + kOffRing, kStageBytes, 1024);  // MN-major ring
+  const uint64_t dP = sw128_desc(sbase + kOffP, 16, 1024);               // K-major P
+  constexpr uint32_t kSlotDesc = kStageBytes >> 4;
 
-  auto take = [&](uint32_t& slot) -> bool {
-    slot = n % kStages;
-    if (!wait_bar(bars.ring_full(slot), (n / kStages) & 1, abort_flag)) return false;
-    tc_fence_after();
-    ++n;
-    return true;
+  // A ring slot is filled by TMA, whose completion the barrier itself orders
+  // before the MMA's shared-memory reads: no tcgen05 fence is needed here.
+  // full_parity bit s = parity of this issuer's next phase on slot s
+  uint32_t full_parity = 0;
+  auto take = [&](uint32_t slot_n) -> bool {
+    const uint32_t slot = slot_n % kStages;
+    const bool ok = wait_bar(bars.ring_full(slot, role), (full_parity >> slot) & 1u, abort_flag);
+    full_parity ^= 1u << slot;
+    return ok;
   };
 
   while (seg_next(p, cl, cur, s)) {
     const int nunits = (s.t_hi - s.t_lo) * p.nsh;
     if (nunits == 0) continue;
-    if (!wait_bar(bars.q_full(), qloads & 1, abort_flag)) return;
-    tc_fence_after();
+    if (qk) {
+      if (!wait_bar(bars.q_full(), qloads & 1, abort_flag)) return;
+      tc_fence_after();
+    }
     ++qloads;
     for (int j = 0; j <= nunits; ++j) {
-      if (j < nunits) {
+      if (j < nunits) {  // QK^T(j): dq + 1 stages
         const uint32_t Ug = U0 + j;
-        const int g = shard_of(p, j % p.nsh);
-        const uint32_t dS = tmem + kColS + 64 * (Ug & 1);
-        uint32_t acc = 0;
-        for (int i = 0; i <= dq; ++i) {
-          const int c = i < dq ? g * dq + i : 8;
-          int k0 = 0, k1 = 4;
-          if (i == dq) rope_steps(p, g, k0, k1);
-          uint32_t slot;
-          if (!take(slot)) return;
-          const uint32_t a0 = sbase + kOffQ + c * kStageBytes;
-          const uint32_t b0 = sbase + kOffRing + slot * kStageBytes;
-          for (int kk = k0; kk < k1; ++kk) {
-            mma_pair_f16(dS, sw128_desc(a0 + 32 * kk, 16, 1024), sw128_desc(b0 + 32 * kk, 16, 1024),
-                         kIdescQK, acc);
-            acc = 1;
-          }
-          mma_commit_pair(bars.ring_empty(slot), 0x3);
-        }
-        mma_commit_pair(bars.s_full(Ug & 1), 0x3);
-        if (j == nunits - 1) mma_commit_pair(bars.q_empty(), 0x3);
-      }
-      if (j >= 1) {
-        const int k = j - 1;
-        const uint32_t Ug = U0 + k;
-        const int g = shard_of(p, k % p.nsh);
-        const bool first = k < p.nsh;  // first tile of this shard in the segment
-        if (!wait_bar(bars.p_full(Ug & 1), (Ug >> 1) & 1, abort_flag)) return;
-        tc_fence_after();
-        const uint32_t pbase = sbase + kOffP + (Ug & 1) * 2 * kStageBytes;
-        for (int nl = 0; nl < p.d / 128; ++nl) {
-          const int ng = g * (p.d / 128) + nl;
-          const uint32_t dO = tmem + kColO + 64 * (ng - ng0);
-          for (int half = 0; half < 2; ++half) {
-            uint32_t slot;
-            if (!take(slot)) return;
-            const uint32_t a0 = pbase + half * kStageBytes;
-            const uint32_t b0 = sbase + kOffRing + slot * kStageBytes;
+        if (qk && (Ug & 1) == parity_role) {
+          const int g = shard_of(p, j % p.nsh);
+          // S[Ug & 1] is free once the softmax of unit Ug - 2 has read it
+          if (Ug >= 2 && !wait_bar(bars.p_full(Ug & 1), ((Ug - 2) >> 1) & 1, abort_flag)) return;
+          tc_fence_after();
+          const uint32_t dS = tmem + kColS + 64 * (Ug & 1);
+          int rk0, rk1;
+          rope_steps(p, g, rk0, rk1);
+          uint32_t acc = 0;
+          for (int i = 0; i <= dq; ++i) {
+            const bool rope = i == dq;
+            const int c = rope ? 8 : g * dq + i;
+            const uint32_t slot = (n + i) % kStages;
+            if (!take(n + i)) return;
+            const uint64_t a = dQ + (uint64_t)(c * kSlotDesc);
+            const uint64_t b = dRk + (uint64_t)(slot * kSlotDesc);
+#pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (first && half == 0 && kk == 0) ? 0u : 1u;
-              mma_pair_f16(dO, sw128_desc(a0 + 32 * kk, 16, 1024),
-                           sw128_desc(b0 + 2048 * kk, kStageBytes, 1024), kIdescPV, acc);
+              if (!rope || (kk >= rk0 && kk < rk1)) {
+                mma_pair_f16(dS, a + 2 * kk, b + 2 * kk, kIdescQK, acc);
+                acc = 1;
+              }
             }
             mma_commit_pair(bars.ring_empty(slot), 0x3);
           }
+          mma_commit_pair(bars.s_full(Ug & 1), 0x3);
         }
-        mma_commit_pair(bars.p_empty(Ug & 1), 0x3);
+        n += dq + 1;
+      }
+      if (j >= 1) {  // PV(j - 1): 2 stages per latent chunk
+        const int k = j - 1;
+        const uint32_t Ug = U0 + k;
+        if (!qk) {
+          const int g = shard_of(p, k % p.nsh);
+          const uint32_t first = k < p.nsh ? 1u : 0u;  // first tile of this shard here
+          if (!wait_bar(bars.p_full(Ug & 1), (Ug >> 1) & 1, abort_flag)) return;
+          tc_fence_after();
+          const uint64_t pa = dP + (uint64_t)((Ug & 1) * 2 * kSlotDesc);
+          for (int nl = nl_lo; nl < nl_hi; ++nl) {
+            const uint32_t dO = tmem + kColO + 64 * (g * nchunks + nl - ng0);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t sn = n + 2 * nl + half;
+              const uint32_t slot = sn % kStages;
+              if (!take(sn)) return;
+              const uint64_t a = pa + (uint64_t)(half * kSlotDesc);
+              const uint64_t b = dRm + (uint64_t)(slot * kSlotDesc);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t acc = (half == 0 && kk == 0) ? (first ^ 1u) : 1u;
+                mma_pair_f16(dO, a + 2 * kk, b + 128 * kk, kIdescPV, acc);
+              }
+              mma_commit_pair(bars.ring_empty(slot), 0x3);
+            }
+          }
+          // both PV roles arrive (count 2): P[Ug & 1] free and O up to date
+          mma_commit_pair(bars.p_empty(Ug & 1), 0x3);
+        }
+        n += 2 * nchunks;
       }
     }
+    // both QK roles arrive on q_empty (count 2) once their QKs of this
+    // segment have completed
+    if (qk) mma_commit_pair(bars.q_empty(), 0x3);
     U0 += nunits;
   }
 }
@@ -555,7 +662,7 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if ((tid & 31) == 0) mbar_arrive_cluster(pf_c[Ug & 1]);
+      if ((tid & 31) == 0) mbar_arrive_remote(pf_c[Ug & 1]);
     }
     U += nunits;
     // epilogue: all PVs of the segment done
@@ -601,24 +708,24 @@ tpla_decode_sm100_kernel(const __grid_constant__ CUtensorMap qmap,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bars.ring_full(s), 1);
+      for (int o = 0; o < 4; ++o) mbar_init(bars.ring_full(s, o), 1);
       mbar_init(bars.ring_empty(s), 1);
     }
     mbar_init(bars.q_full(), 1);
-    mbar_init(bars.q_empty(), 1);
+    mbar_init(bars.q_empty(), 2);   // the two QK issuers
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
       mbar_init(bars.p_full(i), 8);  // 4 softmax warps x 2 CTAs
-      mbar_init(bars.p_empty(i), 1);
+      mbar_init(bars.p_empty(i), 2);  // the two PV issuers
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kWarpProducer0 && lane == 0) {
     tma_prefetch(&qmap);
     tma_prefetch(&kvmap);
   }
-  if (warp == 5) {
+  if (warp == kWarpIssuer0) {
     tmem_alloc_pair(sbase + kOffTmemSlot, kTmemCols);
     tmem_relinquish_pair();
   }
@@ -627,17 +734,18 @@ tpla_decode_sm100_kernel(const __grid_constant__ CUtensorMap qmap,
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemSlot);
 
-  if (warp == 4) {
-    if (lane == 0) producer(p, &qmap, &kvmap, cl, rank, sbase, bars, abort_flag);
-  } else if (warp == 5) {
-    if (lane == 0 && rank == 0) mma_issuer(p, cl, sbase, tmem, bars, abort_flag);
+  if (warp >= kWarpIssuer0) {
+    if (lane == 0 && rank == 0)
+      mma_issuer(p, cl, warp - kWarpIssuer0, sbase, tmem, bars, abort_flag);
+  } else if (warp >= kWarpProducer0) {
+    producer(p, &qmap, &kvmap, cl, warp - kWarpProducer0, rank, sbase, bars, abort_flag);
   } else {
     softmax_warps(p, cl, rank, sbase, smem, tmem, bars, abort_flag);
   }
   __syncwarp();
   tc_fence_before();
   cluster_sync();
-  if (warp == 5) {
+  if (warp == kWarpIssuer0) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, kTmemCols);
   }

@@ -141,9 +141,12 @@ def make_inputs(B: int, H: int, lens, *, paged: bool = True, decay: bool = False
                     meta=dict(seed=seed, decay=decay, paged=paged))
 
 
-def make_workload(name: str, pin: bool = False) -> Workload:
+def make_workload(name: str, pin: bool = False, batch: int | None = None) -> Workload:
+    """A named workload; ``batch`` keeps the per-request recipe with fewer
+    requests (small profiling captures)."""
     c = CONFIGS[name]
-    return make_inputs(c["B"], c["H"], c["lens"], paged=c["paged"],
+    B = c["B"] if batch is None else int(batch)
+    return make_inputs(B, c["H"], c["lens"], paged=c["paged"],
                        decay=c["decay"], seed=c["seed"], wuv=c["wuv"],
                        name=name, pin=pin)
 
