@@ -15,19 +15,26 @@
 //    128-token tiles.  MMA M = 128 heads: CTA r holds heads [64r, 64r + 64)
 //    of Q in shared memory and the rows of S, P and O for those heads in its
 //    tensor memory.  QK^T uses N = 128 tokens, one 64-token page per CTA;
-//    PV uses N = 128 latent columns, 64 from each CTA.
-//  * Tiles are staged by TMA (no multicast) into a ring of 8 KB slots, each
-//    one [64 rows][64 bf16] box with the 128-byte swizzle the MMA reads
-//    directly: K-major for QK^T, the same bytes MN-major for PV.  The PV
-//    columns are fetched again (mostly from L2) because the pair splits QK
-//    by tokens and PV by latent columns.
+//    PV uses N = 256 latent columns (128 from each CTA), the widest pair MMA,
+//    which keeps each SM's tensor pipe at its full rate with a single
+//    issuing thread.
+//  * Tiles are staged by TMA (no multicast) into a ring of eight 16 KB slots.
+//    A 4-D view of the cache (column, row, 64-column chunk, page) lets one
+//    copy land two consecutive [64 rows][64 bf16] chunk tiles with
+//    the 128-byte swizzle the MMA reads directly: K-major for QK^T, the same
+//    bytes MN-major for PV.  A copy takes ~2 us to land under load, so the
+//    ring depth (bytes in flight per SM) sets the bandwidth; four producer
+//    warps keep the slots refilled.  The PV columns are fetched again (mostly
+//    from L2) because the pair splits QK^T by tokens and PV by latent columns.
 //  * TMEM per CTA: two S buffers (64 columns each) and O (256 columns).
 //    Softmax warps read S with tcgen05.ld, keep a running max per shard and
 //    rescale O in TMEM only when the max grows by more than 2^8 (so P stays
 //    below 256 and bf16); P goes to shared memory for the PV MMA.
 //  * TPLA shards are independent attention problems sharing the cache rows:
-//    a (tile, shard) "unit" is one QK^T, one softmax and one PV, pipelined
-//    two deep (S and P double-buffered).
+//    a (tile, shard) "unit" is one QK^T, one softmax and one PV.  S is
+//    double-buffered in TMEM; P has one shared-memory buffer (the ring gets
+//    the space).  Three issuing threads: QK^T of even units, QK^T of odd
+//    units, PV.  Two softmax warpgroups split each unit's tokens.
 //  * Split-KV: a persistent grid of one pair per two SMs walks a balanced
 //    range of the concatenated (request, tile) sequence; requests cut by a
 //    range boundary leave normalised partials + lse in the workspace and
@@ -53,14 +60,20 @@ namespace {
 using namespace ptx;
 
 constexpr int kTileTok = 128;      // tokens per tile (two pages)
-constexpr int kStageBytes = 8192;  // one [64][64] bf16 box
-constexpr int kProducers = 4;      // TMA-issuing warps
-constexpr int kStages = 12;        // TMA ring depth (a multiple of kProducers)
+constexpr int kChunkBytes = 8192;  // one [64 rows][64 bf16] chunk tile
+constexpr int kSlotChunks = 2;     // chunk tiles per ring slot
+constexpr int kSlotBytes = kSlotChunks * kChunkBytes;
+constexpr int kSlots = 8;          // ring depth
+constexpr int kProducers = 4;      // slot s is filled by producer warp s % kProducers
+constexpr int kPBufs = 1;          // P tiles in shared memory
+static_assert(kSlots % kProducers == 0, "each ring slot belongs to one producer");
 constexpr int kQChunks = 9;        // 576 / 64 column chunks of q
-constexpr int kWarpProducer0 = 4;  // warps 0-3 softmax, 4-7 producers, 8-11 MMA issuers
+constexpr int kRopeChunk = 8;      // chunk index of the 64 rope columns
+constexpr int kRoles = 3;          // MMA issuers: QK^T of even units, of odd units, PV
+constexpr int kSoftmaxWarps = 8;   // two warpgroups
+constexpr int kWarpProducer0 = kSoftmaxWarps;  // warps 0-7 softmax, 8-11 producers, 12-14 MMA issuers
 constexpr int kWarpIssuer0 = kWarpProducer0 + kProducers;
-constexpr int kThreads = 32 * (kWarpIssuer0 + 4);
-static_assert(kStages % kProducers == 0, "each ring slot belongs to one producer");
+constexpr int kThreads = 32 * (kWarpIssuer0 + kRoles);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // S buffers: [0, 64), [64, 128)
 constexpr uint32_t kColO = 128;    // O: [128, 384)
@@ -69,20 +82,22 @@ constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 constexpr int kOffQ = 0;
-constexpr int kOffP = kOffQ + kQChunks * kStageBytes;
-constexpr int kOffRing = kOffP + 4 * kStageBytes;
-constexpr int kOffBar = kOffRing + kStages * kStageBytes;
-constexpr int kNumBars = 5 * kStages + 8;  // full[4][kStages], empty[kStages], 8 more
+constexpr int kOffP = kOffQ + kQChunks * kChunkBytes;
+constexpr int kOffRing = kOffP + kPBufs * 2 * kChunkBytes;
+constexpr int kOffBar = kOffRing + kSlots * kSlotBytes;
+constexpr int kNumBars = (kRoles + 1) * kSlots + 10;  // full[role][slot], empty[slot], 10 more
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemSlot + 4;
-constexpr int kOffXbuf = kOffAbort + 12;           // float [2][128]
-constexpr int kOffLbuf = kOffXbuf + 2 * 128 * 4;   // float [128][4]
-constexpr int kSmemUsed = kOffLbuf + 128 * 4 * 4;
+constexpr int kOffXbuf = kOffAbort + 12;              // float [2][2][128]
+constexpr int kOffLbuf = kOffXbuf + 2 * 2 * 128 * 4;  // float [2][128][4]
+constexpr int kSmemUsed = kOffLbuf + 2 * 128 * 4 * 4;
 constexpr int kSmemBytes = kSmemUsed + 1024;       // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffRing % 1024 == 0 && kSlotBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
+constexpr uint32_t kIdescPV256 = idesc_bf16_f32(128, 256, false, true);
+constexpr uint32_t kIdescPV128 = idesc_bf16_f32(128, 128, false, true);
 
 __device__ int g_status;
 
@@ -96,6 +111,9 @@ struct Params {
   int cap_tokens;   // tokens one request's cache can hold
   int paged;
   int B, H, G, split_rope, shard, nsh, d;
+  int dq;    // latent 64-column chunks per shard (d / 64)
+  int NB;    // PV block width: min(256, d) latent columns per MMA
+  int nblk;  // PV blocks per shard (d / NB)
   float scale_log2;  // softmax scale * log2(e)
   void* out;
   int out_bf16;
@@ -208,6 +226,29 @@ __device__ __forceinline__ void rope_steps(const Params& p, int g, int& k0, int&
   }
 }
 
+// Stage plan of one unit (tile t, shard g), shared by producers and issuers
+// so that both walk the same stage sequence.
+//  QK^T: the shard's latent chunks g*dq .. g*dq + dq - 1 followed by the rope
+//        chunk, packed kSlotChunks per stage in that order; item i of a stage
+//        sits at byte offset 8 KB * i of its slot.
+//  PV:   items (block j, page pg), j-major.  An item is this CTA's half of
+//        latent block j (NB/128 chunks) for the 64 tokens of page pg; one item
+//        per stage when NB = 256, the two pages of the block when NB = 128.
+__device__ __forceinline__ int qk_nstages(const Params& p) {
+  return (p.dq + 1 + kSlotChunks - 1) / kSlotChunks;
+}
+__device__ __forceinline__ int qk_item_chunk(const Params& p, int g, int item) {
+  return item < p.dq ? g * p.dq + item : kRopeChunk;
+}
+__device__ __forceinline__ int pv_items_per_stage(const Params& p) { return p.NB == 256 ? 1 : 2; }
+__device__ __forceinline__ int pv_nstages(const Params& p) {
+  return 2 * p.nblk / pv_items_per_stage(p);
+}
+// first chunk of CTA `rank`'s half of latent block j of shard g
+__device__ __forceinline__ int pv_chunk(const Params& p, int g, int j, uint32_t rank) {
+  return g * p.dq + j * (p.NB / 64) + (int)rank * (p.NB / 128);
+}
+
 // ---------------------------------------------------------------- waits
 
 // Bounded wait.  The bound uses the SM cycle counter: reading %globaltimer
@@ -244,55 +285,70 @@ __device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity,
 // full barrier per (slot, issuer) every barrier has a single consumer that
 // takes its phases strictly in order.
 struct Bars {
+  static constexpr int kX = (kRoles + 1) * kSlots;
   uint32_t base;
-  __device__ uint32_t ring_full(int s, int owner) const { return base + 8 * (owner * kStages + s); }
-  __device__ uint32_t ring_empty(int s) const { return base + 8 * (4 * kStages + s); }
-  __device__ uint32_t q_full() const { return base + 8 * (5 * kStages); }
-  __device__ uint32_t q_empty() const { return base + 8 * (5 * kStages + 1); }
-  __device__ uint32_t s_full(int i) const { return base + 8 * (5 * kStages + 2 + i); }
-  __device__ uint32_t p_full(int i) const { return base + 8 * (5 * kStages + 4 + i); }
-  __device__ uint32_t p_empty(int i) const { return base + 8 * (5 * kStages + 6 + i); }
+  __device__ uint32_t ring_full(int s, int role) const { return base + 8 * (role * kSlots + s); }
+  __device__ uint32_t ring_empty(int s) const { return base + 8 * (kRoles * kSlots + s); }
+  __device__ uint32_t q_full() const { return base + 8 * kX; }
+  __device__ uint32_t q_empty() const { return base + 8 * (kX + 1); }
+  __device__ uint32_t s_full(int i) const { return base + 8 * (kX + 2 + i); }
+  __device__ uint32_t p_full(int i) const { return base + 8 * (kX + 4 + i); }
+  __device__ uint32_t p_empty(int i) const { return base + 8 * (kX + 6 + i); }
+  __device__ uint32_t s_free(int i) const { return base + 8 * (kX + 8 + i); }
 };
 
 // ---------------------------------------------------------------- producer
 
-// Physical block ids of one request, fetched 32 pages at a time by the
-// whole producer warp (one coalesced load) and handed to lane 0 by shuffle,
-// so TMA issue never waits on a page-table load.
+// Physical block ids of one request, 32 pages per window.  Each lane of the
+// producer warp holds one entry of three consecutive windows (prev, cur,
+// next): stages of the previous tile still hit after the window advanced,
+// and advancing issues the load of the window after next, which is not read
+// until the producer gets there 32 pages later.  So TMA issue never waits
+// on a page-table load except at the start of a request.
 struct PageWindow {
-  int b = -1, base = 0, blk = 0;
+  int b = -1, base = 0;
+  int prev = 0, cur = 0, next = 0;
+
+  __device__ static int raw(const Params& p, const Segment& s, int pg, int npages) {
+    return (pg >= 0 && pg < npages) ? p.page_table[(int64_t)s.b * p.pt_sb + pg] : p.num_blocks;
+  }
 
   __device__ int get(const Params& p, const Segment& s, int page, int lane) {
     const int npages = (s.L + 63) / 64;
     if (page >= npages) return p.num_blocks;  // beyond the request: reads as zeros
-    if (s.b != b || page < base || page >= base + 32) {
+    const int wb = page & ~31;
+    if (s.b != b || wb < base - 32 || wb > base + 32) {
       b = s.b;
-      base = page;
-      const int pg = base + lane;
-      int v = p.num_blocks;
-      if (pg < npages) {
-        v = p.page_table[(int64_t)s.b * p.pt_sb + pg];
-        if (v < 0 || v >= p.num_blocks) {
-          set_status(TPLA_ERR_DEVICE_BOUNDS);
-          v = p.num_blocks;
-        }
-      }
-      blk = v;
+      base = wb;
+      prev = raw(p, s, base - 32 + lane, npages);
+      cur = raw(p, s, base + lane, npages);
+      next = raw(p, s, base + 32 + lane, npages);
+    } else if (wb == base + 32) {
+      prev = cur;
+      cur = next;
+      base = wb;
+      next = raw(p, s, base + 32 + lane, npages);
     }
-    return __shfl_sync(0xffffffffu, blk, page - base);
+    // wb is now base or base - 32; `next` is not touched, so its load stays in flight
+    int blk = __shfl_sync(0xffffffffu, wb == base ? cur : prev, page & 31);
+    if (blk < 0 || blk >= p.num_blocks) {
+      set_status(TPLA_ERR_DEVICE_BOUNDS);
+      blk = p.num_blocks;
+    }
+    return blk;
   }
 };
 
 // Runs on all 32 lanes of the producer warp (uniform control flow); lane 0
 // issues the barrier arrivals and TMA copies.
 //
-// A thread issuing TMA copies waits a few hundred cycles per copy, so one
-// producer cannot feed the pipeline: kProducers warps share the stage
-// sequence, stage n being loaded by warp n % kProducers.  kStages is a
-// multiple of kProducers, so every ring slot (and its empty barrier) always
-// belongs to the same producer, which takes its phases in order.
-__device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtensorMap* kvmap,
-                         int cl, int pid, uint32_t rank, uint32_t sbase, const Bars& bars,
+// A thread's TMA copies complete one after another, so the ring has one
+// producer warp per slot: stage n goes to slot n % kSlots and is loaded by
+// warp (n % kSlots) % kProducers, which therefore takes the phases of its slots' empty
+// barrier strictly in order.
+__device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtensorMap* kv1,
+                         const CUtensorMap* kv2, int cl, int pid,
+                         uint32_t rank, uint32_t sbase, const Bars& bars,
                          volatile int* abort_flag) {
   const int lane = threadIdx.x & 31;
   const bool leader_lane = lane == 0;
@@ -302,33 +358,31 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
   PageWindow win;
   uint32_t n = 0, qloads = 0, U0 = 0;
   const uint32_t q_full_c = mapa(bars.q_full(), 0);
-  const int dq = p.d / 64;  // latent chunks per shard
-  const int hsplit = (p.d / 128 + 1) / 2;  // PV chunks [0, hsplit) -> issuer 2, rest -> 3
+  const int nq = qk_nstages(p), np = pv_nstages(p), ipst = pv_items_per_stage(p);
+  const int pv_k = p.NB / 128;  // chunks per PV item
 
-  // Stage n goes to slot n % kStages once the slot's previous stage was
-  // released, and signals the full barrier of its consuming issuer `owner`.
-  // Returns 1 when this warp loads stage n, 0 when another producer does,
-  // -1 on abort.  Warp-uniform.
-  auto next_slot = [&](uint32_t& slot, uint32_t& full_c, int owner) -> int {
+  // Claims stage n.  Returns 1 when this warp loads it (slot free, the
+  // leader CTA's full barrier of consumer `owner` armed for `bytes` per CTA),
+  // 0 when another producer does, -1 on abort.  Warp-uniform.
+  auto next_slot = [&](uint32_t& slot, uint32_t& full_c, int owner, uint32_t bytes) -> int {
     const uint32_t me = n++;
-    if (me % kProducers != (uint32_t)pid) return 0;
-    slot = me % kStages;
-    if (me >= (uint32_t)kStages) {
-      if (!wait_bar_warp(bars.ring_empty(slot), ((me / kStages) - 1) & 1, abort_flag))
-        return -1;
+    slot = me % kSlots;
+    if (slot % kProducers != (uint32_t)pid) return 0;
+    if (me >= (uint32_t)kSlots) {
+      if (!wait_bar_warp(bars.ring_empty(slot), ((me / kSlots) - 1) & 1, abort_flag)) return -1;
     }
     full_c = mapa(bars.ring_full(slot, owner), 0);
-    if (rank == 0 && leader_lane)
-      mbar_arrive_expect_tx(bars.ring_full(slot, owner), 2 * kStageBytes);
+    if (rank == 0 && leader_lane) mbar_arrive_expect_tx(bars.ring_full(slot, owner), 2 * bytes);
     return 1;
   };
-  auto load_kv = [&](uint32_t slot, uint32_t full_c, int chunk, int t, int half) {
-    const uint32_t dst = sbase + kOffRing + slot * kStageBytes;
+  // k consecutive chunk tiles from `chunk` of page pg (0/1) of tile t
+  auto load = [&](uint32_t dst, uint32_t full_c, int chunk, int k, int t, int pg) {
+    const CUtensorMap* map = k == 1 ? kv1 : kv2;
     if (p.paged) {
-      const int blk = win.get(p, s, 2 * t + half, lane);
-      if (leader_lane) tma_load_3d_pair(dst, kvmap, 64 * chunk, 0, blk, full_c);
+      const int blk = win.get(p, s, 2 * t + pg, lane);
+      if (leader_lane) tma_load_4d_pair(dst, map, 0, 0, chunk, blk, full_c);
     } else if (leader_lane) {
-      tma_load_3d_pair(dst, kvmap, 64 * chunk, kTileTok * t + 64 * half, s.b, full_c);
+      tma_load_4d_pair(dst, map, 0, kTileTok * t + 64 * pg, chunk, s.b, full_c);
     }
   };
 
@@ -337,41 +391,53 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
     if (nunits == 0) continue;
     if (pid == 0) {  // q of this segment, once its previous user is done
       if (qloads > 0 && !wait_bar_warp(bars.q_empty(), (qloads - 1) & 1, abort_flag)) return;
-      const int nq = p.shard < 0 ? kQChunks : dq + 1;
+      const int nqc = p.shard < 0 ? kQChunks : p.dq + 1;
       if (leader_lane) {
-        if (rank == 0) mbar_arrive_expect_tx(bars.q_full(), 2 * nq * kStageBytes);
-        for (int i = 0; i < nq; ++i) {
-          const int c = p.shard < 0 ? i : (i < dq ? p.shard * dq + i : 8);
-          tma_load_3d_pair(sbase + kOffQ + c * kStageBytes, qmap, 64 * c, 64 * (int)rank, s.b,
+        if (rank == 0) mbar_arrive_expect_tx(bars.q_full(), 2 * nqc * kChunkBytes);
+        for (int i = 0; i < nqc; ++i) {
+          const int c = p.shard < 0 ? i : qk_item_chunk(p, p.shard, i);
+          tma_load_3d_pair(sbase + kOffQ + c * kChunkBytes, qmap, 64 * c, 64 * (int)rank, s.b,
                            q_full_c);
         }
       }
     }
     ++qloads;
     for (int j = 0; j <= nunits; ++j) {
-      if (j < nunits) {  // QK^T stages of unit j: this CTA's page, shard columns
+      if (j < nunits) {  // QK^T stages of unit j: this CTA's page, shard columns + rope
         const int t = s.t_lo + j / p.nsh;
         const int g = shard_of(p, j % p.nsh);
         const int owner = (int)((U0 + j) & 1);
-        for (int i = 0; i <= dq; ++i) {
-          const int c = i < dq ? g * dq + i : 8;
+        for (int st = 0; st < nq; ++st) {
+          const int lo = st * kSlotChunks, hi = min(lo + kSlotChunks, p.dq + 1);
           uint32_t slot, full_c;
-          const int r = next_slot(slot, full_c, owner);
+          const int r = next_slot(slot, full_c, owner, (uint32_t)(hi - lo) * kChunkBytes);
           if (r < 0) return;
-          if (r > 0) load_kv(slot, full_c, c, t, (int)rank);
+          if (r == 0) continue;
+          const uint32_t base = sbase + kOffRing + slot * kSlotBytes;
+          // one copy per run of consecutive chunk indices
+          for (int i = lo; i < hi;) {
+            const int c0 = qk_item_chunk(p, g, i);
+            int k = 1;
+            while (i + k < hi && qk_item_chunk(p, g, i + k) == c0 + k) ++k;
+            load(base + (i - lo) * kChunkBytes, full_c, c0, k, t, (int)rank);
+            i += k;
+          }
         }
       }
       if (j >= 1) {  // PV stages of unit j-1: both pages, this CTA's latent half
         const int k = j - 1;
         const int t = s.t_lo + k / p.nsh;
         const int g = shard_of(p, k % p.nsh);
-        for (int nl = 0; nl < p.d / 128; ++nl) {
-          const int ng = g * (p.d / 128) + nl;
-          for (int half = 0; half < 2; ++half) {
-            uint32_t slot, full_c;
-            const int r = next_slot(slot, full_c, nl < hsplit ? 2 : 3);
-            if (r < 0) return;
-            if (r > 0) load_kv(slot, full_c, 2 * ng + (int)rank, t, half);
+        for (int st = 0; st < np; ++st) {
+          uint32_t slot, full_c;
+          const int r = next_slot(slot, full_c, 2, (uint32_t)(ipst * pv_k) * kChunkBytes);
+          if (r < 0) return;
+          if (r == 0) continue;
+          const uint32_t base = sbase + kOffRing + slot * kSlotBytes;
+          for (int i = 0; i < ipst; ++i) {
+            const int it = st * ipst + i;
+            load(base + i * pv_k * kChunkBytes, full_c, pv_chunk(p, g, it >> 1, rank), pv_k, t,
+                 it & 1);
           }
         }
       }
@@ -382,15 +448,14 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
 
 // ---------------------------------------------------------------- MMA issuers
 //
-// One thread issuing tcgen05.mma waits ~150 cycles per instruction whatever
-// its shape, while a 128 x 128 x 16 pair MMA keeps the tensor pipe busy for
-// only 32 cycles per SM.  So four warps of the leader CTA issue MMAs into
-// independent accumulators: role 0/1 = QK^T of even/odd units (S buffer
-// Ug & 1), role 2/3 = PV of the first/second half of the unit's 128-wide
-// latent chunks (disjoint O columns).  Every issuer walks the producer's
-// stage sequence and consumes (waits for, multiplies, releases) only its
-// own ring slots; a commit tracks only the issuing thread's MMAs, so each
-// issuer releases its own slots and signals its own barriers.
+// One thread can issue a tcgen05.mma about every 55 cycles, while a
+// 128 x 128 x 16 pair MMA (QK^T) keeps the tensor pipe busy for only 32
+// cycles per SM; a 128 x 256 x 16 one (PV) for 64.  So three threads of the
+// leader CTA issue MMAs into independent accumulators: role 0/1 = QK^T of
+// even/odd units (S buffer Ug & 1), role 2 = PV.  Every issuer walks the
+// producers' stage sequence and consumes (waits for, multiplies, releases)
+// only its own ring stages; a commit tracks only the issuing thread's MMAs,
+// so each issuer releases its own slots and signals its own barriers.
 
 __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, uint32_t tmem,
                            const Bars& bars, volatile int* abort_flag) {
@@ -398,30 +463,26 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
   seg_begin(p, cl, cur);
   Segment s;
   uint32_t n = 0, qloads = 0, U0 = 0;
-  const int dq = p.d / 64;
-  const int nchunks = p.d / 128;
-  const int ng0 = p.shard < 0 ? 0 : p.shard * nchunks;
   const bool qk = role < 2;
-  const uint32_t parity_role = (uint32_t)(role & 1);
-  // PV roles split the unit's latent chunks: [0, h) and [h, nchunks)
-  const int hsplit = (nchunks + 1) / 2;
-  const int nl_lo = role == 2 ? 0 : hsplit;
-  const int nl_hi = role == 2 ? hsplit : nchunks;
+  const int nq = qk_nstages(p), np = pv_nstages(p), ipst = pv_items_per_stage(p);
+  const int g0 = p.shard < 0 ? 0 : p.shard;
+  const uint32_t idesc_pv = p.NB == 256 ? kIdescPV256 : kIdescPV128;
+  const uint32_t pv_item_desc = (uint32_t)((p.NB / 128) * kChunkBytes) >> 4;
   // Descriptor templates; an operand at byte offset `o` from a region start
   // is template + (o >> 4) (shared memory is below 256 KB, so the 14-bit
   // start-address field never overflows).
   const uint64_t dQ = sw128_desc(sbase + kOffQ, 16, 1024);               // K-major q
   const uint64_t dRk = sw128_desc(sbase + kOffRing, 16, 1024);           // K-major ring
-  const uint64_t dRm = sw128_desc(sbase + kOffRing, kStageBytes, 1024);  // MN-major ring
+  const uint64_t dRm = sw128_desc(sbase + kOffRing, kChunkBytes, 1024);  // MN-major ring
   const uint64_t dP = sw128_desc(sbase + kOffP, 16, 1024);               // K-major P
-  constexpr uint32_t kSlotDesc = kStageBytes >> 4;
+  constexpr uint32_t kChunkDesc = kChunkBytes >> 4;
+  constexpr uint32_t kSlotDesc = kSlotBytes >> 4;
 
   // A ring slot is filled by TMA, whose completion the barrier itself orders
   // before the MMA's shared-memory reads: no tcgen05 fence is needed here.
   // full_parity bit s = parity of this issuer's next phase on slot s
   uint32_t full_parity = 0;
-  auto take = [&](uint32_t slot_n) -> bool {
-    const uint32_t slot = slot_n % kStages;
+  auto take = [&](uint32_t slot) -> bool {
     const bool ok = wait_bar(bars.ring_full(slot, role), (full_parity >> slot) & 1u, abort_flag);
     full_parity ^= 1u << slot;
     return ok;
@@ -436,67 +497,69 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
     }
     ++qloads;
     for (int j = 0; j <= nunits; ++j) {
-      if (j < nunits) {  // QK^T(j): dq + 1 stages
+      if (j < nunits) {  // QK^T(j)
         const uint32_t Ug = U0 + j;
-        if (qk && (Ug & 1) == parity_role) {
+        if (qk && (Ug & 1) == (uint32_t)role) {
           const int g = shard_of(p, j % p.nsh);
           // S[Ug & 1] is free once the softmax of unit Ug - 2 has read it
-          if (Ug >= 2 && !wait_bar(bars.p_full(Ug & 1), ((Ug - 2) >> 1) & 1, abort_flag)) return;
+          if (Ug >= 2 && !wait_bar(bars.s_free(Ug & 1), ((Ug - 2) >> 1) & 1, abort_flag)) return;
           tc_fence_after();
           const uint32_t dS = tmem + kColS + 64 * (Ug & 1);
           int rk0, rk1;
           rope_steps(p, g, rk0, rk1);
           uint32_t acc = 0;
-          for (int i = 0; i <= dq; ++i) {
-            const bool rope = i == dq;
-            const int c = rope ? 8 : g * dq + i;
-            const uint32_t slot = (n + i) % kStages;
-            if (!take(n + i)) return;
-            const uint64_t a = dQ + (uint64_t)(c * kSlotDesc);
-            const uint64_t b = dRk + (uint64_t)(slot * kSlotDesc);
+          for (int st = 0; st < nq; ++st) {
+            const uint32_t slot = (n + st) % kSlots;
+            if (!take(slot)) return;
+            const int lo = st * kSlotChunks, hi = min(lo + kSlotChunks, p.dq + 1);
+            for (int i = lo; i < hi; ++i) {
+              const bool rope = i == p.dq;
+              const uint64_t a = dQ + (uint64_t)(qk_item_chunk(p, g, i) * kChunkDesc);
+              const uint64_t b = dRk + (uint64_t)(slot * kSlotDesc + (i - lo) * kChunkDesc);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              if (!rope || (kk >= rk0 && kk < rk1)) {
-                mma_pair_f16(dS, a + 2 * kk, b + 2 * kk, kIdescQK, acc);
-                acc = 1;
+              for (int kk = 0; kk < 4; ++kk) {
+                if (!rope || (kk >= rk0 && kk < rk1)) {
+                  mma_pair_f16(dS, a + 2 * kk, b + 2 * kk, kIdescQK, acc);
+                  acc = 1;
+                }
               }
             }
             mma_commit_pair(bars.ring_empty(slot), 0x3);
           }
           mma_commit_pair(bars.s_full(Ug & 1), 0x3);
         }
-        n += dq + 1;
+        n += nq;
       }
-      if (j >= 1) {  // PV(j - 1): 2 stages per latent chunk
+      if (j >= 1) {  // PV(j - 1)
         const int k = j - 1;
         const uint32_t Ug = U0 + k;
         if (!qk) {
           const int g = shard_of(p, k % p.nsh);
           const uint32_t first = k < p.nsh ? 1u : 0u;  // first tile of this shard here
-          if (!wait_bar(bars.p_full(Ug & 1), (Ug >> 1) & 1, abort_flag)) return;
+          if (!wait_bar(bars.p_full(Ug % kPBufs), (Ug / kPBufs) & 1, abort_flag)) return;
           tc_fence_after();
-          const uint64_t pa = dP + (uint64_t)((Ug & 1) * 2 * kSlotDesc);
-          for (int nl = nl_lo; nl < nl_hi; ++nl) {
-            const uint32_t dO = tmem + kColO + 64 * (g * nchunks + nl - ng0);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const uint32_t sn = n + 2 * nl + half;
-              const uint32_t slot = sn % kStages;
-              if (!take(sn)) return;
-              const uint64_t a = pa + (uint64_t)(half * kSlotDesc);
-              const uint64_t b = dRm + (uint64_t)(slot * kSlotDesc);
+          const uint64_t pa = dP + (uint64_t)((Ug % kPBufs) * 2 * kChunkDesc);
+          for (int st = 0; st < np; ++st) {
+            const uint32_t slot = (n + st) % kSlots;
+            if (!take(slot)) return;
+            for (int i = 0; i < ipst; ++i) {
+              const int it = st * ipst + i;
+              const int jb = it >> 1, pg = it & 1;
+              const uint32_t dO = tmem + kColO + ((g - g0) * p.nblk + jb) * (p.NB / 2);
+              const uint64_t a = pa + (uint64_t)(pg * kChunkDesc);
+              const uint64_t b = dRm + (uint64_t)(slot * kSlotDesc + i * pv_item_desc);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t acc = (half == 0 && kk == 0) ? (first ^ 1u) : 1u;
-                mma_pair_f16(dO, a + 2 * kk, b + 128 * kk, kIdescPV, acc);
+                const uint32_t acc = (pg == 0 && kk == 0) ? (first ^ 1u) : 1u;
+                mma_pair_f16(dO, a + 2 * kk, b + 128 * kk, idesc_pv, acc);
               }
-              mma_commit_pair(bars.ring_empty(slot), 0x3);
             }
+            mma_commit_pair(bars.ring_empty(slot), 0x3);
           }
-          // both PV roles arrive (count 2): P[Ug & 1] free and O up to date
-          mma_commit_pair(bars.p_empty(Ug & 1), 0x3);
+          // P[Ug % kPBufs] free and O up to date
+          mma_commit_pair(bars.p_empty(Ug % kPBufs), 0x3);
         }
-        n += 2 * nchunks;
+        n += np;
       }
     }
     // both QK roles arrive on q_empty (count 2) once their QKs of this
@@ -549,19 +612,35 @@ __device__ __forceinline__ void write_lse(const Params& p, const Segment& s, int
   }
 }
 
+// Two warpgroups share each unit: thread (wg, lane) holds TMEM lane `lane`
+// (head 64*rank + lane % 64, token half lane / 64) and tokens
+// [32 wg, 32 wg + 32) of that half.  Both warpgroups keep the same running
+// max (they exchange partial maxima every unit) and each its partial sum;
+// they split the O columns for rescaling and the epilogue.
 __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t sbase,
                               uint8_t* smem, uint32_t tmem, const Bars& bars,
                               volatile int* abort_flag) {
-  const int tid = threadIdx.x;  // 0..127 = TMEM lane
-  const int warp = tid >> 5;
-  const int half = tid >> 6, hl = tid & 63;
+  const int tid = threadIdx.x;  // 0..255
+  const int wg = tid >> 7, lt = tid & 127;
+  const int half = lt >> 6, hl = lt & 63;
   const int head = 64 * (int)rank + hl;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-  float* xbuf = reinterpret_cast<float*>(smem + kOffXbuf);
-  float* lbuf = reinterpret_cast<float*>(smem + kOffLbuf);
+  const uint32_t lane_base = (uint32_t)(32 * ((tid >> 5) & 3)) << 16;
+  float* xbuf = reinterpret_cast<float*>(smem + kOffXbuf);  // [2 buffers][2 wg][128]
+  float* lbuf = reinterpret_cast<float*>(smem + kOffLbuf);  // [2 wg][128][4]
   const uint32_t pf_c[2] = {mapa(bars.p_full(0), 0), mapa(bars.p_full(1), 0)};
-  const int ng0 = p.shard < 0 ? 0 : p.shard * (p.d / 128);
-  const int nchunks = p.d / 128;
+  const uint32_t sf_c[2] = {mapa(bars.s_free(0), 0), mapa(bars.s_free(1), 0)};
+  // O of shard g, block jb: TMEM columns o_col(g, jb) + [0, NB/2); lanes
+  // 0-63 hold latent columns jb*NB + [0, NB/2) of the shard, lanes 64-127
+  // the next NB/2 (the pair MMA's accumulator layout for M = 128).  Pieces
+  // of 32 columns alternate between the warpgroups.
+  const int g0 = p.shard < 0 ? 0 : p.shard;
+  const int npiece = p.NB / 64;  // 32-column pieces per lane and block
+  auto o_col = [&](int g, int jb) -> uint32_t {
+    return kColO + (uint32_t)(((g - g0) * p.nblk + jb) * (p.NB / 2));
+  };
+  auto out_col = [&](int g, int jb) -> int {
+    return (p.shard < 0 ? g * p.d : 0) + jb * p.NB + half * (p.NB / 2);
+  };
 
   Cursor cur;
   seg_begin(p, cl, cur);
@@ -575,13 +654,9 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       for (int j = 0; j < 32; ++j) z[j] = 0.f;
       for (int i = 0; i < p.nsh; ++i) {
         const int g = shard_of(p, i);
-        for (int nl = 0; nl < nchunks; ++nl) {
-          const int ng = g * nchunks + nl;
-          const int col = (p.shard < 0 ? 128 * ng : 128 * nl) + 64 * half;
-          write_out_row(p, s, head, col, z, 0.f);
-          write_out_row(p, s, head, col + 32, z, 0.f);
-        }
-        if (half == 0) write_lse(p, s, head, i, -INFINITY);
+        for (int pc = wg; pc < p.nblk * npiece; pc += 2)
+          write_out_row(p, s, head, out_col(g, pc / npiece) + 32 * (pc % npiece), z, 0.f);
+        if (half == 0 && wg == 0) write_lse(p, s, head, i, -INFINITY);
       }
       continue;
     }
@@ -594,22 +669,33 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       const int t = s.t_lo + k / p.nsh;
       if (!wait_bar(bars.s_full(Ug & 1), (Ug >> 1) & 1, abort_flag)) return;
       tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tmem + lane_base + kColS + 64 * (Ug & 1), r0);
-      tmem_ld32(tmem + lane_base + kColS + 64 * (Ug & 1) + 32, r1);
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_base + kColS + 64 * (Ug & 1) + 32 * wg, r);
       tmem_wait_ld();
-      const int nv = max(0, min(64, s.L - (kTileTok * t + 64 * half)));
-      float x[64];
-      float mx = -INFINITY;
+      // S[Ug & 1] is in registers: let QK^T of unit Ug + 2 overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive_remote(sf_c[Ug & 1]);
+      // raw scores; the positive scale is applied inside the exponent
+      const int nv = max(0, min(32, s.L - (kTileTok * t + 64 * half + 32 * wg)));
+      float x[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        x[j] = j < nv ? __uint_as_float(r0[j]) * p.scale_log2 : -INFINITY;
-        x[j + 32] = j + 32 < nv ? __uint_as_float(r1[j]) * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, fmaxf(x[j], x[j + 32]));
+      for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(r[j]);
+      if (nv < 32) {  // warp-uniform: a warp covers one 32-token range
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = j < nv ? x[j] : -INFINITY;
       }
-      xbuf[(Ug & 1) * 128 + tid] = mx;
-      named_bar_sync(1, 128);
-      mx = fmaxf(mx, xbuf[(Ug & 1) * 128 + (tid ^ 64)]);
+      float mx0 = fmaxf(x[0], x[1]), mx1 = fmaxf(x[2], x[3]);
+#pragma unroll
+      for (int j = 4; j < 32; j += 4) {
+        mx0 = fmaxf(mx0, fmaxf(x[j], x[j + 1]));
+        mx1 = fmaxf(mx1, fmaxf(x[j + 2], x[j + 3]));
+      }
+      float mx = fmaxf(mx0, mx1) * p.scale_log2;
+      float* xb = xbuf + (Ug & 1) * 256;
+      xb[wg * 128 + lt] = mx;
+      named_bar_sync(1, 256);
+      mx = fmaxf(fmaxf(xb[lt], xb[128 + lt]), fmaxf(xb[lt ^ 64], xb[128 + (lt ^ 64)]));
       float mi = m[i];
       float factor = 1.f;
       int resc = 0;
@@ -624,71 +710,70 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       l[i] *= factor;
       if (__any_sync(0xffffffffu, resc)) {
         // O of this shard was last written by an earlier PV: wait for all
-        // issued PVs (up to unit Ug - 1), then rescale in TMEM
-        if (!wait_bar(bars.p_empty((Ug - 1) & 1), ((Ug - 1) >> 1) & 1, abort_flag)) return;
+        // issued PVs (up to unit Ug - 1), then rescale this warpgroup's pieces
+        if (!wait_bar(bars.p_empty((Ug - 1) % kPBufs), ((Ug - 1) / kPBufs) & 1, abort_flag)) return;
         tc_fence_after();
-        for (int nl = 0; nl < nchunks; ++nl) {
-          const int ng = g * nchunks + nl;
-          for (int c2 = 0; c2 < 2; ++c2) {
-            const uint32_t ta = tmem + lane_base + kColO + 64 * (ng - ng0) + 32 * c2;
-            uint32_t o[32];
-            tmem_ld32(ta, o);
-            tmem_wait_ld();
+        for (int pc = wg; pc < p.nblk * npiece; pc += 2) {
+          const uint32_t ta = tmem + lane_base + o_col(g, pc / npiece) + 32 * (pc % npiece);
+          uint32_t o[32];
+          tmem_ld32(ta, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * factor);
-            tmem_st32(ta, o);
-          }
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * factor);
+          tmem_st32(ta, o);
         }
         tmem_wait_st();
       }
       // P = 2^(x - m) in bf16 (masked tokens give 0); l sums the rounded values
-      uint32_t pk[32];
-      float lsum = 0.f;
+      uint32_t pk[16];
+      float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(ex2(x[2 * j] - mi), ex2(x[2 * j + 1] - mi));
+      for (int j = 0; j < 16; ++j) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(ex2(fmaf(x[2 * j], p.scale_log2, -mi)),
+                                                  ex2(fmaf(x[2 * j + 1], p.scale_log2, -mi)));
         float2 f2 = __bfloat1622float2(h2);
-        lsum += f2.x + f2.y;
+        ls0 += f2.x;
+        ls1 += f2.y;
         pk[j] = *reinterpret_cast<uint32_t*>(&h2);
       }
-      l[i] += lsum;
-      if (Ug >= 2) {
-        if (!wait_bar(bars.p_empty(Ug & 1), ((Ug - 2) >> 1) & 1, abort_flag)) return;
+      l[i] += ls0 + ls1;
+      if (Ug >= (uint32_t)kPBufs) {  // P[Ug % kPBufs] was read by PV of unit Ug - kPBufs
+        if (!wait_bar(bars.p_empty(Ug % kPBufs), ((Ug - kPBufs) / kPBufs) & 1, abort_flag)) return;
       }
-      const uint32_t prow = sbase + kOffP + (Ug & 1) * 2 * kStageBytes + half * kStageBytes + hl * 128;
+      // P tile of page `half`: row hl, 16-byte chunks [4 wg, 4 wg + 4), swizzled
+      const uint32_t prow = sbase + kOffP + (Ug % kPBufs) * 2 * kChunkBytes + half * kChunkBytes + hl * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_shared_v4(prow + ((c ^ (hl & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      for (int c = 0; c < 4; ++c)
+        st_shared_v4(prow + (((4 * wg + c) ^ (hl & 7)) << 4), pk[4 * c], pk[4 * c + 1],
+                     pk[4 * c + 2], pk[4 * c + 3]);
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if ((tid & 31) == 0) mbar_arrive_remote(pf_c[Ug & 1]);
+      if ((tid & 31) == 0) mbar_arrive_remote(pf_c[Ug % kPBufs]);
     }
     U += nunits;
     // epilogue: all PVs of the segment done
-    if (!wait_bar(bars.p_empty((U - 1) & 1), ((U - 1) >> 1) & 1, abort_flag)) return;
+    if (!wait_bar(bars.p_empty((U - 1) % kPBufs), ((U - 1) / kPBufs) & 1, abort_flag)) return;
     tc_fence_after();
-    for (int i = 0; i < p.nsh; ++i) lbuf[tid * 4 + i] = l[i];
-    named_bar_sync(1, 128);
+    for (int i = 0; i < p.nsh; ++i) lbuf[(wg * 128 + lt) * 4 + i] = l[i];
+    named_bar_sync(1, 256);
     for (int i = 0; i < p.nsh; ++i) {
       const int g = shard_of(p, i);
-      const float lt = l[i] + lbuf[(tid ^ 64) * 4 + i];
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      const float lse = lt > 0.f ? (m[i] + log2f(lt)) * kLn2 : -INFINITY;
-      for (int nl = 0; nl < nchunks; ++nl) {
-        const int ng = g * nchunks + nl;
-        const int col = (p.shard < 0 ? 128 * ng : 128 * nl) + 64 * half;
-        for (int c2 = 0; c2 < 2; ++c2) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + kColO + 64 * (ng - ng0) + 32 * c2, o);
-          tmem_wait_ld();
-          write_out_row(p, s, head, col + 32 * c2, reinterpret_cast<const float*>(o), inv);
-        }
+      const float lt_sum = (lbuf[lt * 4 + i] + lbuf[(128 + lt) * 4 + i]) +
+                           (lbuf[(lt ^ 64) * 4 + i] + lbuf[(128 + (lt ^ 64)) * 4 + i]);
+      const float inv = lt_sum > 0.f ? 1.f / lt_sum : 0.f;
+      const float lse = lt_sum > 0.f ? (m[i] + log2f(lt_sum)) * kLn2 : -INFINITY;
+      for (int pc = wg; pc < p.nblk * npiece; pc += 2) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + o_col(g, pc / npiece) + 32 * (pc % npiece), o);
+        tmem_wait_ld();
+        write_out_row(p, s, head, out_col(g, pc / npiece) + 32 * (pc % npiece),
+                      reinterpret_cast<const float*>(o), inv);
       }
-      if (half == 0) write_lse(p, s, head, i, lse);
+      if (half == 0 && wg == 0) write_lse(p, s, head, i, lse);
     }
     tc_fence_before();
-    named_bar_sync(1, 128);
+    named_bar_sync(1, 256);
   }
 }
 
@@ -696,7 +781,8 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
 
 __global__ void __launch_bounds__(kThreads, 1)
 tpla_decode_sm100_kernel(const __grid_constant__ CUtensorMap qmap,
-                         const __grid_constant__ CUtensorMap kvmap, const Params p) {
+                         const __grid_constant__ CUtensorMap kv1,
+                         const __grid_constant__ CUtensorMap kv2, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -707,23 +793,25 @@ tpla_decode_sm100_kernel(const __grid_constant__ CUtensorMap qmap,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      for (int o = 0; o < 4; ++o) mbar_init(bars.ring_full(s, o), 1);
+    for (int s = 0; s < kSlots; ++s) {
+      for (int o = 0; o < kRoles; ++o) mbar_init(bars.ring_full(s, o), 1);
       mbar_init(bars.ring_empty(s), 1);
     }
     mbar_init(bars.q_full(), 1);
     mbar_init(bars.q_empty(), 2);   // the two QK issuers
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
-      mbar_init(bars.p_full(i), 8);  // 4 softmax warps x 2 CTAs
-      mbar_init(bars.p_empty(i), 2);  // the two PV issuers
+      mbar_init(bars.p_full(i), 2 * kSoftmaxWarps);  // softmax warps of both CTAs
+      mbar_init(bars.p_empty(i), 1);  // the PV issuer
+      mbar_init(bars.s_free(i), 2 * kSoftmaxWarps);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == kWarpProducer0 && lane == 0) {
     tma_prefetch(&qmap);
-    tma_prefetch(&kvmap);
+    tma_prefetch(&kv1);
+    tma_prefetch(&kv2);
   }
   if (warp == kWarpIssuer0) {
     tmem_alloc_pair(sbase + kOffTmemSlot, kTmemCols);
@@ -738,7 +826,7 @@ tpla_decode_sm100_kernel(const __grid_constant__ CUtensorMap qmap,
     if (lane == 0 && rank == 0)
       mma_issuer(p, cl, warp - kWarpIssuer0, sbase, tmem, bars, abort_flag);
   } else if (warp >= kWarpProducer0) {
-    producer(p, &qmap, &kvmap, cl, warp - kWarpProducer0, rank, sbase, bars, abort_flag);
+    producer(p, &qmap, &kv1, &kv2, cl, warp - kWarpProducer0, rank, sbase, bars, abort_flag);
   } else {
     softmax_warps(p, cl, rank, sbase, smem, tmem, bars, abort_flag);
   }
@@ -923,6 +1011,22 @@ bool encode_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, ui
   return r == CUDA_SUCCESS;
 }
 
+// Cache as a 4-D tensor (column within chunk, row, 64-column chunk, page or
+// request): a box of `k` chunks lands k consecutive [64 rows][64 bf16]
+// swizzled tiles.  Rows past `rows` (and pages past `pages`) read as zeros.
+bool encode_kv_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t pages,
+                   uint64_t row_stride_bytes, uint64_t page_stride_bytes, int k) {
+  cuuint64_t dims[4] = {64, rows, (cuuint64_t)kQChunks, pages};
+  cuuint64_t strides[3] = {row_stride_bytes, 128, page_stride_bytes};
+  cuuint32_t box[4] = {64, 64, (cuuint32_t)k, 1};
+  cuuint32_t estride[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                        strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int num_slots(const DecodeProblem& p, int num_splits, int max_clusters) {
   if (num_splits == 0) return 2 * max_clusters;
   if (num_splits == 1) return 0;
@@ -935,6 +1039,8 @@ bool sm100_supported(const DecodeProblem& p, int device) {
   if (device < 0 || device >= 64) return false;
   if (!(p.G == 1 || p.G == 2 || p.G == 4)) return false;
   if (p.H < 1 || p.H > 128) return false;
+  // the kernel takes the row max of raw scores and scales inside exp2
+  if (!(p.scale > 0.f) || !isfinite(p.scale)) return false;
   if (p.cache_rows > (1 << 30) || (p.page_table && p.num_blocks >= (1LL << 31) - 1)) return false;
   if (p.page_table && p.max_pages > (1 << 24)) return false;
   // 16-byte vector stores of out rows
@@ -958,15 +1064,16 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
   cudaGetDevice(&dev);
   const DeviceInfo& d = device_info(dev);
   if (!d.sm100) return cudaErrorNotSupported;
-  CUtensorMap qmap, kvmap;
+  CUtensorMap qmap, kv[2];
   if (!encode_map(&qmap, dp.q, kWidth, dp.H, dp.B, dp.q_sh * 2, dp.q_sb * 2))
     return cudaErrorInvalidValue;
-  if (dp.page_table) {
-    if (!encode_map(&kvmap, dp.cache, kWidth, kBlock, dp.num_blocks, dp.c_s1 * 2, dp.c_s0 * 2))
-      return cudaErrorInvalidValue;
-  } else {
-    if (!encode_map(&kvmap, dp.cache, kWidth, dp.cache_rows, dp.B, dp.c_s1 * 2, dp.c_s0 * 2))
-      return cudaErrorInvalidValue;
+  for (int k = 1; k <= kSlotChunks; ++k) {
+    const bool ok = dp.page_table
+                        ? encode_kv_map(&kv[k - 1], dp.cache, kBlock, dp.num_blocks, dp.c_s1 * 2,
+                                        dp.c_s0 * 2, k)
+                        : encode_kv_map(&kv[k - 1], dp.cache, dp.cache_rows, dp.B, dp.c_s1 * 2,
+                                        dp.c_s0 * 2, k);
+    if (!ok) return cudaErrorInvalidValue;
   }
   Params p{};
   p.seq_lens = dp.seq_lens;
@@ -982,6 +1089,9 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
   p.shard = dp.shard;
   p.nsh = dp.n_shards;
   p.d = kLatent / dp.G;
+  p.dq = p.d / 64;
+  p.NB = p.d < 256 ? p.d : 256;
+  p.nblk = p.d / p.NB;
   p.scale_log2 = (float)((double)dp.scale * 1.4426950408889634);
   p.out = dp.out;
   p.out_bf16 = dp.out_bf16;
@@ -1014,7 +1124,7 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   launch_config(cfg, attr, clusters, stream);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, tpla_decode_sm100_kernel, qmap, kvmap, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tpla_decode_sm100_kernel, qmap, kv[0], kv[1], p);
   count_launch();
   if (e != cudaSuccess) return e;
   if (p.mode == 0 || p.S > 1) {

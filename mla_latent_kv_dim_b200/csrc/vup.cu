@@ -10,6 +10,12 @@
 // reading W_uv (H * 512 * Dv bf16) and out (B * H * 512 f32) once.  Tensor
 // cores (bf16 in, f32 accumulate); an f32 `out` is split into hi + lo bf16
 // terms, so the result keeps about 16 mantissa bits of `out`.
+//
+// The tiled kernel (16-byte aligned operands) gives every CTA a 64 x 64
+// output tile of one head, streams K in chunks of 64 with the next chunk's
+// global loads in flight while the current one is multiplied, and reads
+// fragments with ldmatrix from padded (conflict-free) shared-memory rows.
+// Other layouts take the element-wise kernel.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -127,6 +133,143 @@ vup_kernel(const void* __restrict__ outp, int64_t o_sb, int64_t o_sh,
   }
 }
 
+// ---------------------------------------------------------------- tiled kernel
+
+constexpr int kTM = 64, kTN = 64, kTK = 64;  // CTA tile: rows of B, columns of Dv, K chunk
+constexpr int kTRow = kTK + 8;               // padded smem row (bf16): 144 bytes
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(128)
+vup_tiled_kernel(const void* __restrict__ outp, int64_t o_sb, int64_t o_sh,
+                 const __nv_bfloat16* __restrict__ W, int64_t w_sh, int64_t w_sj,
+                 float* __restrict__ y, int64_t y_sb, int64_t y_sh, int B, int Dv) {
+  __shared__ __align__(16) __nv_bfloat16 a_hi[kTM][kTRow];
+  __shared__ __align__(16) __nv_bfloat16 a_lo[OUT_BF16 ? 1 : kTM][kTRow];
+  __shared__ __align__(16) __nv_bfloat16 w_s[kTK][kTRow];  // [k][n]
+
+  const int m0 = blockIdx.x * kTM, h = blockIdx.y, n0 = blockIdx.z * kTN;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, t4 = lane & 3;
+
+  // per-thread share of one K chunk
+  constexpr int kAVec = OUT_BF16 ? (kTM * kTK / 8) / 128 : (kTM * kTK / 4) / 128;  // 4 or 8
+  constexpr int kWVec = (kTK * kTN / 8) / 128;                                      // 4
+  uint4 ra[kAVec], rw[kWVec];
+
+  auto load_chunk = [&](int k0) {
+#pragma unroll
+    for (int i = 0; i < kAVec; ++i) {
+      const int idx = tid + 128 * i;
+      const int row = OUT_BF16 ? idx / 8 : idx / 16;
+      const int col = OUT_BF16 ? 8 * (idx % 8) : 4 * (idx % 16);
+      const int b = m0 + row;
+      ra[i] = make_uint4(0, 0, 0, 0);
+      if (b < B) {
+        const int64_t off = (int64_t)b * o_sb + (int64_t)h * o_sh + k0 + col;
+        ra[i] = OUT_BF16 ? *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(outp) + off)
+                         : *reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(outp) + off);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kWVec; ++i) {
+      const int idx = tid + 128 * i;
+      const int kr = idx / 8, n = n0 + 8 * (idx % 8);
+      rw[i] = make_uint4(0, 0, 0, 0);
+      if (n < Dv)
+        rw[i] = *reinterpret_cast<const uint4*>(W + (int64_t)h * w_sh + (int64_t)(k0 + kr) * w_sj + n);
+    }
+  };
+  auto store_chunk = [&]() {
+#pragma unroll
+    for (int i = 0; i < kAVec; ++i) {
+      const int idx = tid + 128 * i;
+      if (OUT_BF16) {
+        *reinterpret_cast<uint4*>(&a_hi[idx / 8][8 * (idx % 8)]) = ra[i];
+      } else {
+        const int row = idx / 16, col = 4 * (idx % 16);
+        const float f[4] = {__uint_as_float(ra[i].x), __uint_as_float(ra[i].y),
+                            __uint_as_float(ra[i].z), __uint_as_float(ra[i].w)};
+        uint32_t hi[2], lo[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(f[2 * e]), h1 = __float2bfloat16_rn(f[2 * e + 1]);
+          hi[e] = pack_bf16(h0, h1);
+          lo[e] = pack_bf16(__float2bfloat16_rn(f[2 * e] - __bfloat162float(h0)),
+                            __float2bfloat16_rn(f[2 * e + 1] - __bfloat162float(h1)));
+        }
+        *reinterpret_cast<uint2*>(&a_hi[row][col]) = make_uint2(hi[0], hi[1]);
+        *reinterpret_cast<uint2*>(&a_lo[row][col]) = make_uint2(lo[0], lo[1]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kWVec; ++i) {
+      const int idx = tid + 128 * i;
+      *reinterpret_cast<uint4*>(&w_s[idx / 8][8 * (idx % 8)]) = rw[i];
+    }
+  };
+
+  float acc[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+
+  load_chunk(0);
+  for (int k0 = 0; k0 < kLatent; k0 += kTK) {
+    __syncthreads();  // previous chunk's fragments are read
+    store_chunk();
+    __syncthreads();
+    if (k0 + kTK < kLatent) load_chunk(k0 + kTK);  // in flight during the MMAs below
+#pragma unroll
+    for (int kk = 0; kk < kTK; kk += 16) {
+      const int ar = 16 * warp + (lane & 15), ac = kk + 8 * (lane >> 4);
+      uint32_t ah[4], al[4];
+      ldsm_x4(smem_u32(&a_hi[ar][ac]), ah[0], ah[1], ah[2], ah[3]);
+      if (!OUT_BF16) ldsm_x4(smem_u32(&a_lo[ar][ac]), al[0], al[1], al[2], al[3]);
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {  // two n-tiles of 8 per ldmatrix
+        const int wr = kk + (lane & 7) + 8 * ((lane >> 3) & 1), wc = 16 * np + 8 * (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(smem_u32(&w_s[wr][wc]), b0, b1, b2, b3);
+        mma_bf16_16816(acc[2 * np], ah, b0, b1);
+        mma_bf16_16816(acc[2 * np + 1], ah, b2, b3);
+        if (!OUT_BF16) {
+          mma_bf16_16816(acc[2 * np], al, b0, b1);
+          mma_bf16_16816(acc[2 * np + 1], al, b2, b3);
+        }
+      }
+    }
+  }
+  const int r0 = m0 + 16 * warp + gid;
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    const int c = n0 + 8 * n + 2 * t4;
+    if (c >= Dv) continue;
+    if (r0 < B)
+      *reinterpret_cast<float2*>(y + (int64_t)r0 * y_sb + (int64_t)h * y_sh + c) =
+          make_float2(acc[n][0], acc[n][1]);
+    if (r0 + 8 < B)
+      *reinterpret_cast<float2*>(y + (int64_t)(r0 + 8) * y_sb + (int64_t)h * y_sh + c) =
+          make_float2(acc[n][2], acc[n][3]);
+  }
+}
+
 template <int NT>
 cudaError_t launch_nt(const void* o, int out_bf16, int64_t o_sb, int64_t o_sh,
                       const __nv_bfloat16* W, int64_t w_sh, int64_t w_sj, float* y,
@@ -150,6 +293,23 @@ cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64
                        cudaStream_t stream) {
   if (B == 0 || H == 0 || Dv == 0) return cudaSuccess;
   const __nv_bfloat16* w = reinterpret_cast<const __nv_bfloat16*>(W);
+  const int ovec = out_bf16 ? 8 : 4;  // elements per 16 bytes
+  const bool tiled = (reinterpret_cast<uintptr_t>(out_latent) & 15u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(W) & 15u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(y) & 7u) == 0 && o_sb % ovec == 0 &&
+                     o_sh % ovec == 0 && w_sh % 8 == 0 && w_sj % 8 == 0 && y_sb % 2 == 0 &&
+                     y_sh % 2 == 0;
+  if (tiled) {
+    dim3 grid((B + kTM - 1) / kTM, H, (Dv + kTN - 1) / kTN);
+    if (out_bf16)
+      vup_tiled_kernel<true><<<grid, 128, 0, stream>>>(out_latent, o_sb, o_sh, w, w_sh, w_sj, y,
+                                                       y_sb, y_sh, B, Dv);
+    else
+      vup_tiled_kernel<false><<<grid, 128, 0, stream>>>(out_latent, o_sb, o_sh, w, w_sh, w_sj, y,
+                                                        y_sb, y_sh, B, Dv);
+    count_launch();
+    return cudaGetLastError();
+  }
   switch (Dv) {
 #define TPLA_VUP_CASE(D) \
   case D: return launch_nt<D / 8>(out_latent, out_bf16, o_sb, o_sh, w, w_sh, w_sj, y, y_sb, y_sh, B, H, stream);
