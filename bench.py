@@ -35,6 +35,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from mla_latent_kv_dim_b200.replicas import aggregate_rate, max_over_ranks  # noqa: E402
 from mla_latent_kv_dim_b200.workloads import (LATENT, ROPE, WIDTH, CONFIGS,  # noqa: E402
                                               make_workload)
 
@@ -108,8 +109,13 @@ def recorded_traffic(kernel_name, workload):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """SM clock and throttle reasons sampled during the timed region: NVML
+    every 2 ms when available (a timed region is tens of milliseconds), else
+    nvidia-smi at its 100 ms minimum."""
 
+    # NVML clocks-event reason bits
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap"}
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -117,9 +123,23 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.nvml = None
+        self.samples = []
         self.lines = []
+        self.stop_flag = False
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.hdl = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.hdl, pynvml.NVML_CLOCK_SM)
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -130,11 +150,33 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def _poll(self):
+        n = self.nvml
+        while not self.stop_flag:
+            try:
+                self.samples.append((n.nvmlDeviceGetClockInfo(self.hdl, n.NVML_CLOCK_SM),
+                                     n.nvmlDeviceGetCurrentClocksEventReasons(self.hdl)))
+            except Exception:
+                break
+            time.sleep(0.002)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
     def stop(self):
+        if self.nvml is not None:
+            self.stop_flag = True
+            self.t.join(timeout=2)
+            sm = [float(c) for c, _ in self.samples]
+            reasons = set()
+            for _, r in self.samples:
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        reasons.add(name)
+            return {"sm_mhz": statistics.median(sm) if sm else None,
+                    "sm_max_mhz": float(self.max_mhz), "reasons": sorted(reasons),
+                    "samples": len(sm), "source": "nvml 2 ms"}
         if not self.proc:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         self.proc.terminate()
@@ -159,7 +201,7 @@ class ClockSampler:
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi 100 ms"}
 
 
 def blas_threads():
@@ -322,12 +364,9 @@ def run_ours(args):
         dist.barrier()
     ms = t_start.elapsed_time(t_end)
     dec_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    if dist:
-        tt = torch.tensor([ms, dec_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, dec_ms = float(tt[0]), float(tt[1])
-    t_step = ms / 1e3 / args.steps
-    value = world * bytes_step / t_step / 1e9
+    ms, dec_ms = max_over_ranks([ms, dec_ms], dist, dev)
+    rate, t_step = aggregate_rate(world, bytes_step, ms, args.steps)
+    value = rate / 1e9
     tok_s = world * B / t_step
 
     # ---- end to end through the public API: host q in, host y out
@@ -359,11 +398,8 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
-    if dist:
-        tt = torch.tensor([e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e_ms = float(tt[0])
-    e2e_val = world * bytes_step / (e_ms / 1e3 / args.steps) / 1e9
+    (e_ms,) = max_over_ranks([e_ms], dist, dev)
+    e2e_val = aggregate_rate(world, bytes_step, e_ms, args.steps)[0] / 1e9
     h2d = q.numel() * 2 + seq.numel() * 4 + (pt.numel() * 4 if pt is not None else 0)
     d2h = y.numel() * 4
 

@@ -78,6 +78,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // S buffers: [0, 64), [64, 128)
 constexpr uint32_t kColO = 128;    // O: [128, 384)
 constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s at full clock
+constexpr uint32_t kWaitSleepNs = 100000;  // suspend hint of one barrier poll
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -258,8 +259,8 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 127) == 0) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if ((i & 15) == 0) {
       if (*abort_flag) return false;
       if (clock64() - t0 > kTimeoutCycles) {
         set_status(TPLA_ERR_DEVICE_TIMEOUT);
@@ -571,6 +572,27 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
 
 // ---------------------------------------------------------------- softmax + epilogue
 
+// Four per-shard floats kept in registers: a runtime index into a local
+// array would put it in (slow) local memory.
+struct Reg4 {
+  float v0, v1, v2, v3;
+  __device__ explicit Reg4(float x) : v0(x), v1(x), v2(x), v3(x) {}
+  __device__ float get(int i) const { return i == 0 ? v0 : (i == 1 ? v1 : (i == 2 ? v2 : v3)); }
+  __device__ void set(int i, float x) {
+    v0 = i == 0 ? x : v0;
+    v1 = i == 1 ? x : v1;
+    v2 = i == 2 ? x : v2;
+    v3 = i == 3 ? x : v3;
+  }
+};
+
+// (lo, hi) rounded to a bf16 pair, lo in the low half
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 __device__ __forceinline__ void write_out_row(const Params& p, const Segment& s, int head,
                                               int col0, const float* v, float inv) {
   if (head >= p.H) return;
@@ -660,8 +682,7 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       }
       continue;
     }
-    float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    float l[4] = {0.f, 0.f, 0.f, 0.f};
+    Reg4 m(-INFINITY), l(0.f);
     for (int k = 0; k < nunits; ++k) {
       const uint32_t Ug = U + k;
       const int i = k % p.nsh;
@@ -696,7 +717,7 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       xb[wg * 128 + lt] = mx;
       named_bar_sync(1, 256);
       mx = fmaxf(fmaxf(xb[lt], xb[128 + lt]), fmaxf(xb[lt ^ 64], xb[128 + (lt ^ 64)]));
-      float mi = m[i];
+      float mi = m.get(i);
       float factor = 1.f;
       int resc = 0;
       if (mi == -INFINITY) {
@@ -706,8 +727,8 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
         mi = mx;
         resc = 1;
       }
-      m[i] = mi;
-      l[i] *= factor;
+      m.set(i, mi);
+      l.set(i, l.get(i) * factor);
       if (__any_sync(0xffffffffu, resc)) {
         // O of this shard was last written by an earlier PV: wait for all
         // issued PVs (up to unit Ug - 1), then rescale this warpgroup's pieces
@@ -729,14 +750,13 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(ex2(fmaf(x[2 * j], p.scale_log2, -mi)),
-                                                  ex2(fmaf(x[2 * j + 1], p.scale_log2, -mi)));
-        float2 f2 = __bfloat1622float2(h2);
-        ls0 += f2.x;
-        ls1 += f2.y;
-        pk[j] = *reinterpret_cast<uint32_t*>(&h2);
+        const uint32_t u = cvt_bf16x2(ex2(fmaf(x[2 * j], p.scale_log2, -mi)),
+                                      ex2(fmaf(x[2 * j + 1], p.scale_log2, -mi)));
+        ls0 += __uint_as_float(u << 16);
+        ls1 += __uint_as_float(u & 0xffff0000u);
+        pk[j] = u;
       }
-      l[i] += ls0 + ls1;
+      l.set(i, l.get(i) + (ls0 + ls1));
       if (Ug >= (uint32_t)kPBufs) {  // P[Ug % kPBufs] was read by PV of unit Ug - kPBufs
         if (!wait_bar(bars.p_empty(Ug % kPBufs), ((Ug - kPBufs) / kPBufs) & 1, abort_flag)) return;
       }
@@ -755,14 +775,14 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
     // epilogue: all PVs of the segment done
     if (!wait_bar(bars.p_empty((U - 1) % kPBufs), ((U - 1) / kPBufs) & 1, abort_flag)) return;
     tc_fence_after();
-    for (int i = 0; i < p.nsh; ++i) lbuf[(wg * 128 + lt) * 4 + i] = l[i];
+    for (int i = 0; i < p.nsh; ++i) lbuf[(wg * 128 + lt) * 4 + i] = l.get(i);
     named_bar_sync(1, 256);
     for (int i = 0; i < p.nsh; ++i) {
       const int g = shard_of(p, i);
       const float lt_sum = (lbuf[lt * 4 + i] + lbuf[(128 + lt) * 4 + i]) +
                            (lbuf[(lt ^ 64) * 4 + i] + lbuf[(128 + (lt ^ 64)) * 4 + i]);
       const float inv = lt_sum > 0.f ? 1.f / lt_sum : 0.f;
-      const float lse = lt_sum > 0.f ? (m[i] + log2f(lt_sum)) * kLn2 : -INFINITY;
+      const float lse = lt_sum > 0.f ? (m.get(i) + log2f(lt_sum)) * kLn2 : -INFINITY;
       for (int pc = wg; pc < p.nblk * npiece; pc += 2) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_base + o_col(g, pc / npiece) + 32 * (pc % npiece), o);
