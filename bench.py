@@ -406,7 +406,8 @@ def run_ours(args):
     # ---- roofline of the dominant kernel (decode), live CUDA-event timing
     dec_s = dec_ms / 1e3
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    tc_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    # the timed region is tens of milliseconds at full clock: the burst GEMM peak applies
+    tc_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved_gbs = bytes_step / dec_s / 1e9
     achieved_tf = flops_step / dec_s / 1e12
     t_hbm = bytes_step / (hbm_peak * 1e9)
@@ -425,7 +426,7 @@ def run_ours(args):
                  "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
                  "hbm_gbs": round(achieved_gbs, 1), "hbm_frac": round(achieved_gbs / hbm_peak, 4),
                  "tensor_tflops": round(achieved_tf, 2),
-                 "tensor_frac_sustained": round(achieved_tf / tc_peak, 4),
+                 "tensor_frac_burst": round(achieved_tf / tc_peak, 4),
                  "bytes_per_launch": bytes_step, "flops_per_launch": flops_step,
                  "decode_ms": round(dec_ms, 4)})
 

@@ -19,11 +19,11 @@ Sources (web pages on TPLA / MLA latent-cache sharding):
   "Tests / validation".
 * [ABSTRACT] "TPLA: Tensor Parallel Latent Attention for Efficient
   Disaggregated Prefill & Decode Inference", abstract.
-* [VERDICT] pith.science review of arXiv 2508.15881: skeptic critique
+* [REVIEW] pith.science review of arXiv 2508.15881: skeptic critique
   (load-bearing attack on Eq. 6), referee report (significance; major comments
   on Eq. 22/25), pith extraction (key machinery), desk-editor letter.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 1. Eq. 6 is not printed; the reviewers state it is an *unscaled* local
    softmax.  Shard g therefore uses the same ``scale`` as exact MLA and no
@@ -62,7 +62,7 @@ def shard_columns(G: int, g: int, rope_mode: str = "replicate"):
     """Return (latent_cols, rope_cols) of shard ``g`` out of ``G``.
 
     [ABSTRACT]: TPLA partitions the latent representation and each head's
-    input dimension across devices.  [VERDICT referee_report.significance]:
+    input dimension across devices.  [REVIEW referee_report.significance]:
     the per-device cache is 256 + 64 = 320 dims at TP=2, so the rope part is
     replicated to every shard.  ``split`` (rope also cut into G slices) is
     the alternative reading; contiguous slices in shard order (readings 2, 3).
@@ -186,9 +186,9 @@ def tpla_decode_ref(q, rows, G, rope_mode, scale, shard=None):
     """TPLA decode: G latent shards, an independent softmax per shard.
 
     [ISSUE] "Directions under investigation": each rank runs local attention
-    over its latent slice.  [VERDICT pith_extraction.key_machinery]: device i
+    over its latent slice.  [REVIEW pith_extraction.key_machinery]: device i
     computes softmax(Q_i (cKV_i U)^T) with all query heads replicated;
-    [VERDICT skeptic_critique]: Eq. 6 is an unscaled local softmax.
+    [REVIEW skeptic_critique]: Eq. 6 is an unscaled local softmax.
     Shard g's logits use its latent columns plus its rope columns; its
     values are its latent columns only.  Outputs are concatenated in shard
     order (reading 5).
@@ -220,7 +220,7 @@ def tpla_decode_ref(q, rows, G, rope_mode, scale, shard=None):
 def gla_decode_ref(q, rows, G, rope_mode, scale):
     """TPLA written as Grouped Latent Attention with G*H heads.
 
-    [VERDICT desk_editor.letter / pith_summary]: TPLA is a special case of
+    [REVIEW desk_editor.letter / pith_summary]: TPLA is a special case of
     GLA with replicated heads.  Head (g, h) of the GLA model sees latent group
     g only.  This restatement builds the grouped keys explicitly, evaluates
     all G*H heads in one batched contraction and normalises with SciPy's
@@ -376,7 +376,7 @@ def vup_sharded_ref(out_latent, W_uv, G):
 def per_head_cosine(a, b):
     """Cosine similarity per (request, head) of two [B, H, V] outputs.
 
-    [VERDICT skeptic_critique.concrete_test] proposes the per-head cosine of
+    [REVIEW skeptic_critique.concrete_test] proposes the per-head cosine of
     the TPLA output against exact MLA as the direct fidelity measurement.
     """
     a = np.asarray(a, np.float64)
