@@ -63,10 +63,9 @@ constexpr int kTileTok = 128;      // tokens per tile (two pages)
 constexpr int kChunkBytes = 8192;  // one [64 rows][64 bf16] chunk tile
 constexpr int kSlotChunks = 2;     // chunk tiles per ring slot
 constexpr int kSlotBytes = kSlotChunks * kChunkBytes;
-constexpr int kSlots = 8;          // ring depth
-constexpr int kProducers = 4;      // slot s is filled by producer warp s % kProducers
+constexpr int kRingSlots = 8;      // slots shared by the QK^T ring and the PV ring
+constexpr int kProducers = 4;      // two producer warps per ring
 constexpr int kPBufs = 1;          // P tiles in shared memory
-static_assert(kSlots % kProducers == 0, "each ring slot belongs to one producer");
 constexpr int kQChunks = 9;        // 576 / 64 column chunks of q
 constexpr int kRopeChunk = 8;      // chunk index of the 64 rope columns
 constexpr int kRoles = 3;          // MMA issuers: QK^T of even units, of odd units, PV
@@ -84,9 +83,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 constexpr int kOffQ = 0;
 constexpr int kOffP = kOffQ + kQChunks * kChunkBytes;
-constexpr int kOffRing = kOffP + kPBufs * 2 * kChunkBytes;
-constexpr int kOffBar = kOffRing + kSlots * kSlotBytes;
-constexpr int kNumBars = (kRoles + 1) * kSlots + 10;  // full[role][slot], empty[slot], 10 more
+constexpr int kOffRing = kOffP + kPBufs * 2 * kChunkBytes;  // QK^T slots, then PV slots
+constexpr int kOffBar = kOffRing + kRingSlots * kSlotBytes;
+constexpr int kNumBars = 5 * kRingSlots + 10;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemSlot + 4;
 constexpr int kOffXbuf = kOffAbort + 12;              // float [2][2][128]
@@ -115,6 +114,7 @@ struct Params {
   int dq;    // latent 64-column chunks per shard (d / 64)
   int NB;    // PV block width: min(256, d) latent columns per MMA
   int nblk;  // PV blocks per shard (d / NB)
+  int qk_slots, pv_slots;  // ring split (sum kRingSlots)
   float scale_log2;  // softmax scale * log2(e)
   void* out;
   int out_bf16;
@@ -286,10 +286,13 @@ __device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity,
 // full barrier per (slot, issuer) every barrier has a single consumer that
 // takes its phases strictly in order.
 struct Bars {
-  static constexpr int kX = (kRoles + 1) * kSlots;
+  static constexpr int kX = 5 * kRingSlots;
   uint32_t base;
-  __device__ uint32_t ring_full(int s, int role) const { return base + 8 * (role * kSlots + s); }
-  __device__ uint32_t ring_empty(int s) const { return base + 8 * (kRoles * kSlots + s); }
+  // QK^T ring: one full barrier per (slot, QK issuer), see above
+  __device__ uint32_t qk_full(int s, int role) const { return base + 8 * (role * kRingSlots + s); }
+  __device__ uint32_t qk_empty(int s) const { return base + 8 * (2 * kRingSlots + s); }
+  __device__ uint32_t pv_full(int s) const { return base + 8 * (3 * kRingSlots + s); }
+  __device__ uint32_t pv_empty(int s) const { return base + 8 * (4 * kRingSlots + s); }
   __device__ uint32_t q_full() const { return base + 8 * kX; }
   __device__ uint32_t q_empty() const { return base + 8 * (kX + 1); }
   __device__ uint32_t s_full(int i) const { return base + 8 * (kX + 2 + i); }
@@ -343,16 +346,18 @@ struct PageWindow {
 // Runs on all 32 lanes of the producer warp (uniform control flow); lane 0
 // issues the barrier arrivals and TMA copies.
 //
-// A thread's TMA copies complete one after another, so the ring has one
-// producer warp per slot: stage n goes to slot n % kSlots and is loaded by
-// warp (n % kSlots) % kProducers, which therefore takes the phases of its slots' empty
-// barrier strictly in order.
+// Two rings: QK^T stages and PV stages, each of kRingSlots slots with two
+// producer warps (slot s of a ring is filled by that ring's warp s % 2, which
+// therefore takes the phases of its slots' empty barriers in order).  With
+// separate rings, PV stages waiting for their softmax never hold up the
+// loads of later QK^T stages.
 __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtensorMap* kv1,
-                         const CUtensorMap* kv2, int cl, int pid,
-                         uint32_t rank, uint32_t sbase, const Bars& bars,
-                         volatile int* abort_flag) {
+                         const CUtensorMap* kv2, int cl, int pid, uint32_t rank, uint32_t sbase,
+                         const Bars& bars, volatile int* abort_flag) {
   const int lane = threadIdx.x & 31;
   const bool leader_lane = lane == 0;
+  const bool qk_ring = pid < 2;
+  const uint32_t rpid = (uint32_t)(pid & 1);
   Cursor cur;
   seg_begin(p, cl, cur);
   Segment s;
@@ -361,19 +366,24 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
   const uint32_t q_full_c = mapa(bars.q_full(), 0);
   const int nq = qk_nstages(p), np = pv_nstages(p), ipst = pv_items_per_stage(p);
   const int pv_k = p.NB / 128;  // chunks per PV item
+  const uint32_t nslots = (uint32_t)(qk_ring ? p.qk_slots : p.pv_slots);
+  const uint32_t ring_base = sbase + kOffRing + (qk_ring ? 0u : (uint32_t)p.qk_slots * kSlotBytes);
 
-  // Claims stage n.  Returns 1 when this warp loads it (slot free, the
-  // leader CTA's full barrier of consumer `owner` armed for `bytes` per CTA),
-  // 0 when another producer does, -1 on abort.  Warp-uniform.
+  // Claims stage n of this warp's ring.  Returns 1 when this warp loads it
+  // (slot free, the leader CTA's full barrier of consumer `owner` armed for
+  // `bytes` per CTA), 0 when the ring's other producer does, -1 on abort.
+  // Warp-uniform.
   auto next_slot = [&](uint32_t& slot, uint32_t& full_c, int owner, uint32_t bytes) -> int {
     const uint32_t me = n++;
-    slot = me % kSlots;
-    if (slot % kProducers != (uint32_t)pid) return 0;
-    if (me >= (uint32_t)kSlots) {
-      if (!wait_bar_warp(bars.ring_empty(slot), ((me / kSlots) - 1) & 1, abort_flag)) return -1;
+    slot = me % nslots;
+    if ((slot & 1u) != rpid) return 0;
+    if (me >= nslots) {
+      const uint32_t eb = qk_ring ? bars.qk_empty(slot) : bars.pv_empty(slot);
+      if (!wait_bar_warp(eb, ((me / nslots) - 1) & 1, abort_flag)) return -1;
     }
-    full_c = mapa(bars.ring_full(slot, owner), 0);
-    if (rank == 0 && leader_lane) mbar_arrive_expect_tx(bars.ring_full(slot, owner), 2 * bytes);
+    const uint32_t fb = qk_ring ? bars.qk_full(slot, owner) : bars.pv_full(slot);
+    full_c = mapa(fb, 0);
+    if (rank == 0 && leader_lane) mbar_arrive_expect_tx(fb, 2 * bytes);
     return 1;
   };
   // k consecutive chunk tiles from `chunk` of page pg (0/1) of tile t
@@ -403,10 +413,10 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
       }
     }
     ++qloads;
-    for (int j = 0; j <= nunits; ++j) {
-      if (j < nunits) {  // QK^T stages of unit j: this CTA's page, shard columns + rope
-        const int t = s.t_lo + j / p.nsh;
-        const int g = shard_of(p, j % p.nsh);
+    for (int j = 0; j < nunits; ++j) {
+      const int t = s.t_lo + j / p.nsh;
+      const int g = shard_of(p, j % p.nsh);
+      if (qk_ring) {  // QK^T stages of unit j: this CTA's page, shard columns + rope
         const int owner = (int)((U0 + j) & 1);
         for (int st = 0; st < nq; ++st) {
           const int lo = st * kSlotChunks, hi = min(lo + kSlotChunks, p.dq + 1);
@@ -414,7 +424,7 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
           const int r = next_slot(slot, full_c, owner, (uint32_t)(hi - lo) * kChunkBytes);
           if (r < 0) return;
           if (r == 0) continue;
-          const uint32_t base = sbase + kOffRing + slot * kSlotBytes;
+          const uint32_t base = ring_base + slot * kSlotBytes;
           // one copy per run of consecutive chunk indices
           for (int i = lo; i < hi;) {
             const int c0 = qk_item_chunk(p, g, i);
@@ -424,17 +434,13 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
             i += k;
           }
         }
-      }
-      if (j >= 1) {  // PV stages of unit j-1: both pages, this CTA's latent half
-        const int k = j - 1;
-        const int t = s.t_lo + k / p.nsh;
-        const int g = shard_of(p, k % p.nsh);
+      } else {  // PV stages of unit j: both pages, this CTA's latent half
         for (int st = 0; st < np; ++st) {
           uint32_t slot, full_c;
-          const int r = next_slot(slot, full_c, 2, (uint32_t)(ipst * pv_k) * kChunkBytes);
+          const int r = next_slot(slot, full_c, 0, (uint32_t)(ipst * pv_k) * kChunkBytes);
           if (r < 0) return;
           if (r == 0) continue;
-          const uint32_t base = sbase + kOffRing + slot * kSlotBytes;
+          const uint32_t base = ring_base + slot * kSlotBytes;
           for (int i = 0; i < ipst; ++i) {
             const int it = st * ipst + i;
             load(base + i * pv_k * kChunkBytes, full_c, pv_chunk(p, g, it >> 1, rank), pv_k, t,
@@ -473,8 +479,10 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
   // is template + (o >> 4) (shared memory is below 256 KB, so the 14-bit
   // start-address field never overflows).
   const uint64_t dQ = sw128_desc(sbase + kOffQ, 16, 1024);               // K-major q
-  const uint64_t dRk = sw128_desc(sbase + kOffRing, 16, 1024);           // K-major ring
-  const uint64_t dRm = sw128_desc(sbase + kOffRing, kChunkBytes, 1024);  // MN-major ring
+  const uint32_t nslots = (uint32_t)(qk ? p.qk_slots : p.pv_slots);
+  const uint32_t off_pv = kOffRing + (uint32_t)p.qk_slots * kSlotBytes;
+  const uint64_t dRk = sw128_desc(sbase + kOffRing, 16, 1024);        // K-major QK^T ring
+  const uint64_t dRm = sw128_desc(sbase + off_pv, kChunkBytes, 1024);  // MN-major PV ring
   const uint64_t dP = sw128_desc(sbase + kOffP, 16, 1024);               // K-major P
   constexpr uint32_t kChunkDesc = kChunkBytes >> 4;
   constexpr uint32_t kSlotDesc = kSlotBytes >> 4;
@@ -484,7 +492,8 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
   // full_parity bit s = parity of this issuer's next phase on slot s
   uint32_t full_parity = 0;
   auto take = [&](uint32_t slot) -> bool {
-    const bool ok = wait_bar(bars.ring_full(slot, role), (full_parity >> slot) & 1u, abort_flag);
+    const uint32_t fb = qk ? bars.qk_full(slot, role) : bars.pv_full(slot);
+    const bool ok = wait_bar(fb, (full_parity >> slot) & 1u, abort_flag);
     full_parity ^= 1u << slot;
     return ok;
   };
@@ -510,7 +519,7 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
           rope_steps(p, g, rk0, rk1);
           uint32_t acc = 0;
           for (int st = 0; st < nq; ++st) {
-            const uint32_t slot = (n + st) % kSlots;
+            const uint32_t slot = (n + st) % nslots;
             if (!take(slot)) return;
             const int lo = st * kSlotChunks, hi = min(lo + kSlotChunks, p.dq + 1);
             for (int i = lo; i < hi; ++i) {
@@ -525,11 +534,11 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
                 }
               }
             }
-            mma_commit_pair(bars.ring_empty(slot), 0x3);
+            mma_commit_pair(bars.qk_empty(slot), 0x3);
           }
           mma_commit_pair(bars.s_full(Ug & 1), 0x3);
         }
-        n += nq;
+        if (qk) n += nq;
       }
       if (j >= 1) {  // PV(j - 1)
         const int k = j - 1;
@@ -541,7 +550,7 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
           tc_fence_after();
           const uint64_t pa = dP + (uint64_t)((Ug % kPBufs) * 2 * kChunkDesc);
           for (int st = 0; st < np; ++st) {
-            const uint32_t slot = (n + st) % kSlots;
+            const uint32_t slot = (n + st) % nslots;
             if (!take(slot)) return;
             for (int i = 0; i < ipst; ++i) {
               const int it = st * ipst + i;
@@ -555,12 +564,12 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
                 mma_pair_f16(dO, a + 2 * kk, b + 128 * kk, idesc_pv, acc);
               }
             }
-            mma_commit_pair(bars.ring_empty(slot), 0x3);
+            mma_commit_pair(bars.pv_empty(slot), 0x3);
           }
           // P[Ug % kPBufs] free and O up to date
           mma_commit_pair(bars.p_empty(Ug % kPBufs), 0x3);
         }
-        n += np;
+        if (!qk) n += np;
       }
     }
     // both QK roles arrive on q_empty (count 2) once their QKs of this
@@ -813,9 +822,12 @@ tpla_decode_sm100_kernel(const __grid_constant__ CUtensorMap qmap,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kSlots; ++s) {
-      for (int o = 0; o < kRoles; ++o) mbar_init(bars.ring_full(s, o), 1);
-      mbar_init(bars.ring_empty(s), 1);
+    for (int s = 0; s < kRingSlots; ++s) {
+      mbar_init(bars.qk_full(s, 0), 1);
+      mbar_init(bars.qk_full(s, 1), 1);
+      mbar_init(bars.qk_empty(s), 1);
+      mbar_init(bars.pv_full(s), 1);
+      mbar_init(bars.pv_empty(s), 1);
     }
     mbar_init(bars.q_full(), 1);
     mbar_init(bars.q_empty(), 2);   // the two QK issuers
@@ -1112,6 +1124,10 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
   p.dq = p.d / 64;
   p.NB = p.d < 256 ? p.d : 256;
   p.nblk = p.d / p.NB;
+  // QK^T stages wait ~2 us to land and then only for the tensor core, so
+  // they get most of the ring; PV stages are consumed at the softmax's pace
+  p.qk_slots = dp.G == 1 ? 5 : 6;
+  p.pv_slots = kRingSlots - p.qk_slots;
   p.scale_log2 = (float)((double)dp.scale * 1.4426950408889634);
   p.out = dp.out;
   p.out_bf16 = dp.out_bf16;
