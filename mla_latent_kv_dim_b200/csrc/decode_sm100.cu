@@ -486,6 +486,11 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
   const uint64_t dP = sw128_desc(sbase + kOffP, 16, 1024);               // K-major P
   constexpr uint32_t kChunkDesc = kChunkBytes >> 4;
   constexpr uint32_t kSlotDesc = kSlotBytes >> 4;
+  // 32-bit halves: adding an in-range offset to the low half never carries
+  const uint32_t q_lo = (uint32_t)dQ, q_hi = (uint32_t)(dQ >> 32);
+  const uint32_t rk_lo = (uint32_t)dRk, rk_hi = (uint32_t)(dRk >> 32);
+  const uint32_t rm_lo = (uint32_t)dRm, rm_hi = (uint32_t)(dRm >> 32);
+  const uint32_t p_lo = (uint32_t)dP, p_hi = (uint32_t)(dP >> 32);
 
   // A ring slot is filled by TMA, whose completion the barrier itself orders
   // before the MMA's shared-memory reads: no tcgen05 fence is needed here.
@@ -523,13 +528,17 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
             if (!take(slot)) return;
             const int lo = st * kSlotChunks, hi = min(lo + kSlotChunks, p.dq + 1);
             for (int i = lo; i < hi; ++i) {
-              const bool rope = i == p.dq;
-              const uint64_t a = dQ + (uint64_t)(qk_item_chunk(p, g, i) * kChunkDesc);
-              const uint64_t b = dRk + (uint64_t)(slot * kSlotDesc + (i - lo) * kChunkDesc);
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                if (!rope || (kk >= rk0 && kk < rk1)) {
-                  mma_pair_f16(dS, a + 2 * kk, b + 2 * kk, kIdescQK, acc);
+              const uint32_t a = q_lo + (uint32_t)qk_item_chunk(p, g, i) * kChunkDesc;
+              const uint32_t b = rk_lo + slot * kSlotDesc + (uint32_t)(i - lo) * kChunkDesc;
+              if (i < p.dq) {  // latent chunk: four K-steps of 16 columns
+                mma_pair_f16_lh(dS, a, q_hi, b, rk_hi, kIdescQK, acc);
+                mma_pair_f16_lh(dS, a + 2, q_hi, b + 2, rk_hi, kIdescQK, 1u);
+                mma_pair_f16_lh(dS, a + 4, q_hi, b + 4, rk_hi, kIdescQK, 1u);
+                mma_pair_f16_lh(dS, a + 6, q_hi, b + 6, rk_hi, kIdescQK, 1u);
+                acc = 1;
+              } else {  // rope chunk: this shard's K-steps
+                for (int kk = rk0; kk < rk1; ++kk) {
+                  mma_pair_f16_lh(dS, a + 2 * kk, q_hi, b + 2 * kk, rk_hi, kIdescQK, acc);
                   acc = 1;
                 }
               }
@@ -548,7 +557,7 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
           const uint32_t first = k < p.nsh ? 1u : 0u;  // first tile of this shard here
           if (!wait_bar(bars.p_full(Ug % kPBufs), (Ug / kPBufs) & 1, abort_flag)) return;
           tc_fence_after();
-          const uint64_t pa = dP + (uint64_t)((Ug % kPBufs) * 2 * kChunkDesc);
+          const uint32_t pa = p_lo + (Ug % kPBufs) * 2 * kChunkDesc;
           for (int st = 0; st < np; ++st) {
             const uint32_t slot = (n + st) % nslots;
             if (!take(slot)) return;
@@ -556,13 +565,13 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
               const int it = st * ipst + i;
               const int jb = it >> 1, pg = it & 1;
               const uint32_t dO = tmem + kColO + ((g - g0) * p.nblk + jb) * (p.NB / 2);
-              const uint64_t a = pa + (uint64_t)(pg * kChunkDesc);
-              const uint64_t b = dRm + (uint64_t)(slot * kSlotDesc + i * pv_item_desc);
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t acc = (pg == 0 && kk == 0) ? (first ^ 1u) : 1u;
-                mma_pair_f16(dO, a + 2 * kk, b + 128 * kk, idesc_pv, acc);
-              }
+              const uint32_t a = pa + (uint32_t)pg * kChunkDesc;
+              const uint32_t b = rm_lo + slot * kSlotDesc + (uint32_t)i * pv_item_desc;
+              const uint32_t acc0 = pg == 0 ? (first ^ 1u) : 1u;
+              mma_pair_f16_lh(dO, a, p_hi, b, rm_hi, idesc_pv, acc0);
+              mma_pair_f16_lh(dO, a + 2, p_hi, b + 128, rm_hi, idesc_pv, 1u);
+              mma_pair_f16_lh(dO, a + 4, p_hi, b + 256, rm_hi, idesc_pv, 1u);
+              mma_pair_f16_lh(dO, a + 6, p_hi, b + 384, rm_hi, idesc_pv, 1u);
             }
             mma_commit_pair(bars.pv_empty(slot), 0x3);
           }
@@ -594,6 +603,28 @@ struct Reg4 {
     v3 = i == 3 ? x : v3;
   }
 };
+
+// Packed two-lane float arithmetic (sm_100): one instruction for two
+// values halves the softmax's issue slots for these steps, and those issue
+// slots are shared with the MMA-issuing threads of the same sub-partition.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 
 // (lo, hi) rounded to a bf16 pair, lo in the low half
 __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
@@ -756,15 +787,18 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       }
       // P = 2^(x - m) in bf16 (masked tokens give 0); l sums the rounded values
       uint32_t pk[16];
-      float ls0 = 0.f, ls1 = 0.f;
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-mi, -mi);
+      uint64_t ls2 = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const uint32_t u = cvt_bf16x2(ex2(fmaf(x[2 * j], p.scale_log2, -mi)),
-                                      ex2(fmaf(x[2 * j + 1], p.scale_log2, -mi)));
-        ls0 += __uint_as_float(u << 16);
-        ls1 += __uint_as_float(u & 0xffff0000u);
+        float e0, e1;
+        f2_unpack(f2_fma(f2_pack(x[2 * j], x[2 * j + 1]), sc2, nm2), e0, e1);
+        const uint32_t u = cvt_bf16x2(ex2(e0), ex2(e1));
+        ls2 = f2_add(ls2, f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u)));
         pk[j] = u;
       }
+      float ls0, ls1;
+      f2_unpack(ls2, ls0, ls1);
       l.set(i, l.get(i) + (ls0 + ls1));
       if (Ug >= (uint32_t)kPBufs) {  // P[Ug % kPBufs] was read by PV of unit Ug - kPBufs
         if (!wait_bar(bars.p_empty(Ug % kPBufs), ((Ug - kPBufs) / kPBufs) & 1, abort_flag)) return;

@@ -173,6 +173,24 @@ __device__ __forceinline__ void mma_pair_f16(uint32_t d_tmem, uint64_t adesc, ui
       : "memory");
 }
 
+// The same MMA with each descriptor given as 32-bit halves: the low half
+// (start address and leading offset) varies per operand, the high half is
+// constant per layout.  Fewer issuing instructions per MMA matter because
+// the issuing thread shares its SM sub-partition with busy softmax warps.
+__device__ __forceinline__ void mma_pair_f16_lh(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                                uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %5, p;\n\t}"
+      :
+      : "r"(d_tmem), "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on the barrier at offset `bar` in every CTA of `mask` when all
 // prior tcgen05 operations of this thread have completed.
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t mask) {
