@@ -70,9 +70,13 @@ constexpr int kQChunks = 9;        // 576 / 64 column chunks of q
 constexpr int kRopeChunk = 8;      // chunk index of the 64 rope columns
 constexpr int kRoles = 3;          // MMA issuers: QK^T of even units, of odd units, PV
 constexpr int kSoftmaxWarps = 8;   // two warpgroups
-constexpr int kWarpProducer0 = kSoftmaxWarps;  // warps 0-7 softmax, 8-11 producers, 12-14 MMA issuers
-constexpr int kWarpIssuer0 = kWarpProducer0 + kProducers;
-constexpr int kThreads = 32 * (kWarpIssuer0 + kRoles);
+// Warps 0-2 issue MMAs, 3-6 produce, 7-14 run the softmax.  The issuers take
+// the lowest warp ids, which the warp schedulers favour when several warps
+// of a sub-partition are ready; warp w reaches TMEM lanes 32 (w % 4) + [0, 32).
+constexpr int kWarpIssuer0 = 0;
+constexpr int kWarpProducer0 = kWarpIssuer0 + kRoles;
+constexpr int kWarpSoftmax0 = kWarpProducer0 + kProducers;
+constexpr int kThreads = 32 * (kWarpSoftmax0 + kSoftmaxWarps);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // S buffers: [0, 64), [64, 128)
 constexpr uint32_t kColO = 128;    // O: [128, 384)
@@ -682,7 +686,9 @@ __device__ __forceinline__ void write_lse(const Params& p, const Segment& s, int
 __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t sbase,
                               uint8_t* smem, uint32_t tmem, const Bars& bars,
                               volatile int* abort_flag) {
-  const int tid = threadIdx.x;  // 0..255
+  // tid = 128 * warpgroup + TMEM lane (a warp's lanes are fixed by warp % 4)
+  const int w = (int)(threadIdx.x >> 5);
+  const int tid = ((w - kWarpSoftmax0) >> 2) * 128 + 32 * (w & 3) + (int)(threadIdx.x & 31);
   const int wg = tid >> 7, lt = tid & 127;
   const int half = lt >> 6, hl = lt & 63;
   const int head = 64 * (int)rank + hl;
@@ -888,10 +894,10 @@ tpla_decode_sm100_kernel(const __grid_constant__ CUtensorMap qmap,
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemSlot);
 
-  if (warp >= kWarpIssuer0) {
+  if (warp < kWarpProducer0) {
     if (lane == 0 && rank == 0)
       mma_issuer(p, cl, warp - kWarpIssuer0, sbase, tmem, bars, abort_flag);
-  } else if (warp >= kWarpProducer0) {
+  } else if (warp < kWarpSoftmax0) {
     producer(p, &qmap, &kv1, &kv2, cl, warp - kWarpProducer0, rank, sbase, bars, abort_flag);
   } else {
     softmax_warps(p, cl, rank, sbase, smem, tmem, bars, abort_flag);
