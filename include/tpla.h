@@ -125,6 +125,15 @@ typedef struct {
  * [0, num_blocks) or seq_lens larger than the cache can hold are not read;
  * the kernel records TPLA_ERR_DEVICE_BOUNDS in the device status word
  * (tpla_get_device_status) and treats the missing tokens as absent.
+ *
+ * Precondition: the rows of a request's last page (contiguous mode: of its
+ * last 64-row block inside the cache) past seq_lens[b] must hold finite
+ * values.  The tensor-core path reads whole pages and gives those rows zero
+ * weight after the softmax, and 0 * NaN is NaN.
+ *
+ * Kernel choice (opts->kernel = AUTO): the tcgen05 kernel when the device is
+ * sm_100, G is 1, 2 or 4, H <= 128, scale > 0 and out rows are 16-byte
+ * aligned; the portable kernel otherwise.  Both compute the same function.
  */
 TPLA_API int tpla_decode_ex(const tpla_tensor* q, const tpla_tensor* kv_cache,
                    const tpla_tensor* seq_lens, const tpla_tensor* page_table,
