@@ -59,11 +59,11 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kTileTok = 128;      // tokens per tile (two pages)
+constexpr int kTileTok = 256;      // tokens per tile (four pages, two per CTA)
 constexpr int kChunkBytes = 8192;  // one [64 rows][64 bf16] chunk tile
-constexpr int kSlotChunks = 2;     // chunk tiles per ring slot
+constexpr int kSlotChunks = 2;     // 8 KB chunk tiles per ring slot
 constexpr int kSlotBytes = kSlotChunks * kChunkBytes;
-constexpr int kRingSlots = 8;      // slots shared by the QK^T ring and the PV ring
+constexpr int kRingSlots = 7;      // slots shared by the QK^T ring and the PV ring
 constexpr int kProducers = 4;      // two producer warps per ring
 constexpr int kPBufs = 1;          // P tiles in shared memory
 constexpr int kQChunks = 9;        // 576 / 64 column chunks of q
@@ -78,8 +78,8 @@ constexpr int kWarpProducer0 = kWarpIssuer0 + kRoles;
 constexpr int kWarpSoftmax0 = kWarpProducer0 + kProducers;
 constexpr int kThreads = 32 * (kWarpSoftmax0 + kSoftmaxWarps);
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;      // S buffers: [0, 64), [64, 128)
-constexpr uint32_t kColO = 128;    // O: [128, 384)
+constexpr uint32_t kColS = 0;      // S buffers: [0, 128), [128, 256)
+constexpr uint32_t kColO = 256;    // O: [256, 512)
 constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s at full clock
 constexpr uint32_t kWaitSleepNs = 100000;  // suspend hint of one barrier poll
 constexpr float kLn2 = 0.69314718055994530942f;
@@ -87,7 +87,8 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 constexpr int kOffQ = 0;
 constexpr int kOffP = kOffQ + kQChunks * kChunkBytes;
-constexpr int kOffRing = kOffP + kPBufs * 2 * kChunkBytes;  // QK^T slots, then PV slots
+constexpr int kPTileBytes = 4 * kChunkBytes;  // P: 64 heads x 256 tokens, one [64][64] tile per page
+constexpr int kOffRing = kOffP + kPBufs * kPTileBytes;  // QK^T slots, then PV slots
 constexpr int kOffBar = kOffRing + kRingSlots * kSlotBytes;
 constexpr int kNumBars = 5 * kRingSlots + 10;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
@@ -99,7 +100,7 @@ constexpr int kSmemBytes = kSmemUsed + 1024;       // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffRing % 1024 == 0 && kSlotBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
 
-constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 256, false, false);
 constexpr uint32_t kIdescPV256 = idesc_bf16_f32(128, 256, false, true);
 constexpr uint32_t kIdescPV128 = idesc_bf16_f32(128, 128, false, true);
 
@@ -232,22 +233,23 @@ __device__ __forceinline__ void rope_steps(const Params& p, int g, int& k0, int&
 }
 
 // Stage plan of one unit (tile t, shard g), shared by producers and issuers
-// so that both walk the same stage sequence.
-//  QK^T: the shard's latent chunks g*dq .. g*dq + dq - 1 followed by the rope
-//        chunk, packed kSlotChunks per stage in that order; item i of a stage
-//        sits at byte offset 8 KB * i of its slot.
-//  PV:   items (block j, page pg), j-major.  An item is this CTA's half of
-//        latent block j (NB/128 chunks) for the 64 tokens of page pg; one item
-//        per stage when NB = 256, the two pages of the block when NB = 128.
-__device__ __forceinline__ int qk_nstages(const Params& p) {
-  return (p.dq + 1 + kSlotChunks - 1) / kSlotChunks;
-}
+// so that both walk the same stage sequence.  A tile is four pages; CTA r
+// holds pages 2r and 2r + 1 for QK^T.
+//  QK^T: one stage per item (the shard's latent chunks g*dq .. g*dq + dq - 1,
+//        then the rope chunk): chunk c of this CTA's two pages, the second
+//        page's [64][64] tile right after the first, so that one descriptor
+//        with an 8-row stride covers the CTA's 128 tokens.
+//  PV:   items (block j, page pg), j-major over pages 0..3 of the tile.  An
+//        item is this CTA's half of latent block j (NB/128 chunks) for the
+//        64 tokens of page pg; one item per stage when NB = 256, two pages
+//        per stage when NB = 128.
+__device__ __forceinline__ int qk_nstages(const Params& p) { return p.dq + 1; }
 __device__ __forceinline__ int qk_item_chunk(const Params& p, int g, int item) {
   return item < p.dq ? g * p.dq + item : kRopeChunk;
 }
 __device__ __forceinline__ int pv_items_per_stage(const Params& p) { return p.NB == 256 ? 1 : 2; }
 __device__ __forceinline__ int pv_nstages(const Params& p) {
-  return 2 * p.nblk / pv_items_per_stage(p);
+  return 4 * p.nblk / pv_items_per_stage(p);
 }
 // first chunk of CTA `rank`'s half of latent block j of shard g
 __device__ __forceinline__ int pv_chunk(const Params& p, int g, int j, uint32_t rank) {
@@ -390,11 +392,11 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
     if (rank == 0 && leader_lane) mbar_arrive_expect_tx(fb, 2 * bytes);
     return 1;
   };
-  // k consecutive chunk tiles from `chunk` of page pg (0/1) of tile t
+  // k consecutive chunk tiles from `chunk` of page pg (0..3) of tile t
   auto load = [&](uint32_t dst, uint32_t full_c, int chunk, int k, int t, int pg) {
     const CUtensorMap* map = k == 1 ? kv1 : kv2;
     if (p.paged) {
-      const int blk = win.get(p, s, 2 * t + pg, lane);
+      const int blk = win.get(p, s, 4 * t + pg, lane);
       if (leader_lane) tma_load_4d_pair(dst, map, 0, 0, chunk, blk, full_c);
     } else if (leader_lane) {
       tma_load_4d_pair(dst, map, 0, kTileTok * t + 64 * pg, chunk, s.b, full_c);
@@ -423,20 +425,14 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
       if (qk_ring) {  // QK^T stages of unit j: this CTA's page, shard columns + rope
         const int owner = (int)((U0 + j) & 1);
         for (int st = 0; st < nq; ++st) {
-          const int lo = st * kSlotChunks, hi = min(lo + kSlotChunks, p.dq + 1);
           uint32_t slot, full_c;
-          const int r = next_slot(slot, full_c, owner, (uint32_t)(hi - lo) * kChunkBytes);
+          const int r = next_slot(slot, full_c, owner, 2 * kChunkBytes);
           if (r < 0) return;
           if (r == 0) continue;
           const uint32_t base = ring_base + slot * kSlotBytes;
-          // one copy per run of consecutive chunk indices
-          for (int i = lo; i < hi;) {
-            const int c0 = qk_item_chunk(p, g, i);
-            int k = 1;
-            while (i + k < hi && qk_item_chunk(p, g, i + k) == c0 + k) ++k;
-            load(base + (i - lo) * kChunkBytes, full_c, c0, k, t, (int)rank);
-            i += k;
-          }
+          const int c = qk_item_chunk(p, g, st);
+          load(base, full_c, c, 1, t, 2 * (int)rank);
+          load(base + kChunkBytes, full_c, c, 1, t, 2 * (int)rank + 1);
         }
       } else {  // PV stages of unit j: both pages, this CTA's latent half
         for (int st = 0; st < np; ++st) {
@@ -447,8 +443,8 @@ __device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtenso
           const uint32_t base = ring_base + slot * kSlotBytes;
           for (int i = 0; i < ipst; ++i) {
             const int it = st * ipst + i;
-            load(base + i * pv_k * kChunkBytes, full_c, pv_chunk(p, g, it >> 1, rank), pv_k, t,
-                 it & 1);
+            load(base + i * pv_k * kChunkBytes, full_c, pv_chunk(p, g, it >> 2, rank), pv_k, t,
+                 it & 3);
           }
         }
       }
@@ -523,17 +519,17 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
           // S[Ug & 1] is free once the softmax of unit Ug - 2 has read it
           if (Ug >= 2 && !wait_bar(bars.s_free(Ug & 1), ((Ug - 2) >> 1) & 1, abort_flag)) return;
           tc_fence_after();
-          const uint32_t dS = tmem + kColS + 64 * (Ug & 1);
+          const uint32_t dS = tmem + kColS + 128 * (Ug & 1);
           int rk0, rk1;
           rope_steps(p, g, rk0, rk1);
           uint32_t acc = 0;
           for (int st = 0; st < nq; ++st) {
             const uint32_t slot = (n + st) % nslots;
             if (!take(slot)) return;
-            const int lo = st * kSlotChunks, hi = min(lo + kSlotChunks, p.dq + 1);
-            for (int i = lo; i < hi; ++i) {
+            {
+              const int i = st;
               const uint32_t a = q_lo + (uint32_t)qk_item_chunk(p, g, i) * kChunkDesc;
-              const uint32_t b = rk_lo + slot * kSlotDesc + (uint32_t)(i - lo) * kChunkDesc;
+              const uint32_t b = rk_lo + slot * kSlotDesc;
               if (i < p.dq) {  // latent chunk: four K-steps of 16 columns
                 mma_pair_f16_lh(dS, a, q_hi, b, rk_hi, kIdescQK, acc);
                 mma_pair_f16_lh(dS, a + 2, q_hi, b + 2, rk_hi, kIdescQK, 1u);
@@ -561,13 +557,13 @@ __device__ void mma_issuer(const Params& p, int cl, int role, uint32_t sbase, ui
           const uint32_t first = k < p.nsh ? 1u : 0u;  // first tile of this shard here
           if (!wait_bar(bars.p_full(Ug % kPBufs), (Ug / kPBufs) & 1, abort_flag)) return;
           tc_fence_after();
-          const uint32_t pa = p_lo + (Ug % kPBufs) * 2 * kChunkDesc;
+          const uint32_t pa = p_lo + (Ug % kPBufs) * (kPTileBytes >> 4);
           for (int st = 0; st < np; ++st) {
             const uint32_t slot = (n + st) % nslots;
             if (!take(slot)) return;
             for (int i = 0; i < ipst; ++i) {
               const int it = st * ipst + i;
-              const int jb = it >> 1, pg = it & 1;
+              const int jb = it >> 2, pg = it & 3;
               const uint32_t dO = tmem + kColO + ((g - g0) * p.nblk + jb) * (p.NB / 2);
               const uint32_t a = pa + (uint32_t)pg * kChunkDesc;
               const uint32_t b = rm_lo + slot * kSlotDesc + (uint32_t)i * pv_item_desc;
@@ -736,25 +732,30 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       const int t = s.t_lo + k / p.nsh;
       if (!wait_bar(bars.s_full(Ug & 1), (Ug >> 1) & 1, abort_flag)) return;
       tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32(tmem + lane_base + kColS + 64 * (Ug & 1) + 32 * wg, r);
+      // this thread's 64 tokens: page 2 * half + wg of the tile
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tmem + lane_base + kColS + 128 * (Ug & 1) + 64 * wg, r0);
+      tmem_ld32(tmem + lane_base + kColS + 128 * (Ug & 1) + 64 * wg + 32, r1);
       tmem_wait_ld();
       // S[Ug & 1] is in registers: let QK^T of unit Ug + 2 overwrite it
       tc_fence_before();
       __syncwarp();
       if ((tid & 31) == 0) mbar_arrive_remote(sf_c[Ug & 1]);
       // raw scores; the positive scale is applied inside the exponent
-      const int nv = max(0, min(32, s.L - (kTileTok * t + 64 * half + 32 * wg)));
-      float x[32];
+      const int nv = max(0, min(64, s.L - (kTileTok * t + 128 * half + 64 * wg)));
+      float x[64];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(r[j]);
-      if (nv < 32) {  // warp-uniform: a warp covers one 32-token range
+      for (int j = 0; j < 32; ++j) {
+        x[j] = __uint_as_float(r0[j]);
+        x[j + 32] = __uint_as_float(r1[j]);
+      }
+      if (nv < 64) {  // warp-uniform: a warp covers one 64-token range
 #pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = j < nv ? x[j] : -INFINITY;
+        for (int j = 0; j < 64; ++j) x[j] = j < nv ? x[j] : -INFINITY;
       }
       float mx0 = fmaxf(x[0], x[1]), mx1 = fmaxf(x[2], x[3]);
 #pragma unroll
-      for (int j = 4; j < 32; j += 4) {
+      for (int j = 4; j < 64; j += 4) {
         mx0 = fmaxf(mx0, fmaxf(x[j], x[j + 1]));
         mx1 = fmaxf(mx1, fmaxf(x[j + 2], x[j + 3]));
       }
@@ -792,11 +793,11 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
         tmem_wait_st();
       }
       // P = 2^(x - m) in bf16 (masked tokens give 0); l sums the rounded values
-      uint32_t pk[16];
+      uint32_t pk[32];
       const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-mi, -mi);
       uint64_t ls2 = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < 32; ++j) {
         float e0, e1;
         f2_unpack(f2_fma(f2_pack(x[2 * j], x[2 * j + 1]), sc2, nm2), e0, e1);
         const uint32_t u = cvt_bf16x2(ex2(e0), ex2(e1));
@@ -809,12 +810,13 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       if (Ug >= (uint32_t)kPBufs) {  // P[Ug % kPBufs] was read by PV of unit Ug - kPBufs
         if (!wait_bar(bars.p_empty(Ug % kPBufs), ((Ug - kPBufs) / kPBufs) & 1, abort_flag)) return;
       }
-      // P tile of page `half`: row hl, 16-byte chunks [4 wg, 4 wg + 4), swizzled
-      const uint32_t prow = sbase + kOffP + (Ug % kPBufs) * 2 * kChunkBytes + half * kChunkBytes + hl * 128;
+      // P tile of page 2 * half + wg: row hl, all eight 16-byte chunks, swizzled
+      const uint32_t prow = sbase + kOffP + (Ug % kPBufs) * kPTileBytes +
+                            (2 * half + wg) * kChunkBytes + hl * 128;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        st_shared_v4(prow + (((4 * wg + c) ^ (hl & 7)) << 4), pk[4 * c], pk[4 * c + 1],
-                     pk[4 * c + 2], pk[4 * c + 3]);
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(prow + ((c ^ (hl & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                     pk[4 * c + 3]);
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -1166,7 +1168,7 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
   p.nblk = p.d / p.NB;
   // QK^T stages wait ~2 us to land and then only for the tensor core, so
   // they get most of the ring; PV stages are consumed at the softmax's pace
-  p.qk_slots = dp.G == 1 ? 5 : 6;
+  p.qk_slots = 4;
   p.pv_slots = kRingSlots - p.qk_slots;
   p.scale_log2 = (float)((double)dp.scale * 1.4426950408889634);
   p.out = dp.out;
