@@ -1168,7 +1168,8 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
   p.nblk = p.d / p.NB;
   // QK^T stages wait ~2 us to land and then only for the tensor core, so
   // they get most of the ring; PV stages are consumed at the softmax's pace
-  p.qk_slots = 4;
+  // measured: G=1 (eight PV stages per tile) wants the deeper PV ring
+  p.qk_slots = dp.G == 1 ? 3 : 4;
   p.pv_slots = kRingSlots - p.qk_slots;
   p.scale_log2 = (float)((double)dp.scale * 1.4426950408889634);
   p.out = dp.out;
