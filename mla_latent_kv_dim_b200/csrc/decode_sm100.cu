@@ -12,21 +12,21 @@
 //
 // Design (B200):
 //  * A CTA pair (cluster of 2, tcgen05 cta_group::2) owns one stream of
-//    128-token tiles.  MMA M = 128 heads: CTA r holds heads [64r, 64r + 64)
-//    of Q in shared memory and the rows of S, P and O for those heads in its
-//    tensor memory.  QK^T uses N = 128 tokens, one 64-token page per CTA;
-//    PV uses N = 256 latent columns (128 from each CTA), the widest pair MMA,
-//    which keeps each SM's tensor pipe at its full rate with a single
-//    issuing thread.
-//  * Tiles are staged by TMA (no multicast) into a ring of eight 16 KB slots.
-//    A 4-D view of the cache (column, row, 64-column chunk, page) lets one
-//    copy land two consecutive [64 rows][64 bf16] chunk tiles with
-//    the 128-byte swizzle the MMA reads directly: K-major for QK^T, the same
-//    bytes MN-major for PV.  A copy takes ~2 us to land under load, so the
-//    ring depth (bytes in flight per SM) sets the bandwidth; four producer
-//    warps keep the slots refilled.  The PV columns are fetched again (mostly
-//    from L2) because the pair splits QK^T by tokens and PV by latent columns.
-//  * TMEM per CTA: two S buffers (64 columns each) and O (256 columns).
+//    256-token tiles (four pages; CTA r holds pages 2r, 2r + 1 for QK^T).
+//    MMA M = 128 heads: CTA r holds heads [64r, 64r + 64) of Q in shared
+//    memory and the rows of S, P and O for those heads in its tensor memory.
+//    QK^T and PV both use N = 256 (tokens / latent columns, half from each
+//    CTA), the widest pair MMA: each MMA keeps the SM's tensor pipe busy for
+//    64 cycles, longer than one thread needs to issue it.
+//  * Tiles are staged by TMA (no multicast) into seven 16 KB slots, split
+//    into a QK^T ring and a PV ring with two producer warps each.  A 4-D
+//    view of the cache (column, row, 64-column chunk, page) lands [64 rows]
+//    [64 bf16] chunk tiles with the 128-byte swizzle the MMA reads directly:
+//    K-major for QK^T, the same bytes MN-major for PV.  A copy takes ~2 us
+//    to land under load, so the ring depth (bytes in flight per SM) sets the
+//    bandwidth.  The PV columns are fetched again (mostly from L2) because
+//    the pair splits QK^T by tokens and PV by latent columns.
+//  * TMEM per CTA: two S buffers (128 columns each) and O (256 columns).
 //    Softmax warps read S with tcgen05.ld, keep a running max per shard and
 //    rescale O in TMEM only when the max grows by more than 2^8 (so P stays
 //    below 256 and bf16); P goes to shared memory for the PV MMA.
@@ -35,6 +35,9 @@
 //    double-buffered in TMEM; P has one shared-memory buffer (the ring gets
 //    the space).  Three issuing threads: QK^T of even units, QK^T of odd
 //    units, PV.  Two softmax warpgroups split each unit's tokens.
+//  * The issuing threads share their SM sub-partitions with softmax warps
+//    and lose issue slots to them; the MMA issue code is kept short and the
+//    issuers run on the lowest warp ids.
 //  * Split-KV: a persistent grid of one pair per two SMs walks a balanced
 //    range of the concatenated (request, tile) sequence; requests cut by a
 //    range boundary leave normalised partials + lse in the workspace and
