@@ -253,6 +253,17 @@ TPLA_API int tpla_get_device_status(tpla_stream_t stream, int* status);
 TPLA_API int64_t tpla_launch_count(void);
 
 /* TPLA_VERSION of the loaded library. */
+/*
+ * tpla_selftest_wait_timeout -- test support for the device failure path;
+ * the pages have no counterpart.  Launches one thread that waits, through
+ * the same bounded barrier wait the decode kernels use, on a barrier that
+ * nothing completes.  After about `microseconds` (1 .. 1e6) of SM clock the
+ * wait gives up, records TPLA_ERR_DEVICE_TIMEOUT in the device status word
+ * and the kernel returns; the context stays usable.  Read the status with
+ * tpla_get_device_status.  Asynchronous on `stream`.
+ */
+TPLA_API int tpla_selftest_wait_timeout(int microseconds, tpla_stream_t stream);
+
 TPLA_API int tpla_version(void);
 
 #ifdef __cplusplus

@@ -7,7 +7,9 @@ workloads (``workloads``).
 """
 from ._native import (TplaError, decode, decode_simple, decode_workspace_size,  # noqa: F401
                       device_status, error_string, hadamard_apply, launch_count, lse_merge, lib,
+                      selftest_wait_timeout,
                       version, vup_combine)
 
 __all__ = ["TplaError", "decode", "decode_simple", "decode_workspace_size", "device_status",
+           "selftest_wait_timeout",
            "error_string", "hadamard_apply", "launch_count", "lse_merge", "lib", "version", "vup_combine"]

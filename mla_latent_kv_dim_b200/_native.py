@@ -75,9 +75,11 @@ def lib() -> ctypes.CDLL:
             L.tpla_error_string.argtypes = [ctypes.c_int]
             L.tpla_error_string.restype = ctypes.c_char_p
             L.tpla_get_device_status.argtypes = [ctypes.c_void_p, _P(ctypes.c_int)]
+            L.tpla_selftest_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_void_p]
             for f in ("tpla_decode_ex", "tpla_decode", "tpla_decode_workspace_size",
                       "tpla_lse_merge", "tpla_hadamard_apply", "tpla_vup_combine",
-                      "tpla_last_cuda_error", "tpla_get_device_status", "tpla_version"):
+                      "tpla_last_cuda_error", "tpla_get_device_status", "tpla_version",
+                      "tpla_selftest_wait_timeout"):
                 getattr(L, f).restype = ctypes.c_int
             L.tpla_launch_count.restype = ctypes.c_int64
             _lib = L
@@ -227,6 +229,13 @@ def error_string(code: int) -> str:
 def launch_count() -> int:
     """Kernels libtpla has launched in this process so far."""
     return int(lib().tpla_launch_count())
+
+
+def selftest_wait_timeout(microseconds: int = 1000, stream=None) -> None:
+    """Run one bounded barrier wait that nothing completes; the device status
+    then reads TPLA_ERR_DEVICE_TIMEOUT (see tpla_selftest_wait_timeout)."""
+    _check("tpla_selftest_wait_timeout",
+           lib().tpla_selftest_wait_timeout(int(microseconds), _stream(stream)))
 
 
 def version() -> int:

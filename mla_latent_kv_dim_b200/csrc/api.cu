@@ -342,6 +342,19 @@ int tpla_get_device_status(tpla_stream_t stream, int* status) {
   return TPLA_OK;
 }
 
+int tpla_selftest_wait_timeout(int microseconds, tpla_stream_t stream) {
+  if (microseconds < 1 || microseconds > 1000000) return TPLA_ERR_INVALID_ARG;
+  int dev = current_device();
+  int khz = 0;
+  if (cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess || khz <= 0) {
+    cudaGetLastError();
+    khz = 2000000;
+  }
+  const long long cycles = (long long)microseconds * (khz / 1000);
+  cudaError_t e = launch_wait_timeout_selftest(cycles, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
+}
+
 int tpla_version(void) { return TPLA_VERSION; }
 
 int64_t tpla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -264,14 +264,15 @@ __device__ __forceinline__ int pv_chunk(const Params& p, int g, int j, uint32_t 
 // Bounded wait.  The bound uses the SM cycle counter: reading %globaltimer
 // costs about half a microsecond, which would throttle every pipeline
 // hand-off that has to wait.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         long long limit = kTimeoutCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if ((i & 15) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kTimeoutCycles) {
+      if (clock64() - t0 > limit) {
         set_status(TPLA_ERR_DEVICE_TIMEOUT);
         *abort_flag = 1;
         return false;
@@ -1005,6 +1006,23 @@ sm100_merge_kernel(const Params p) {
   }
 }
 
+// ---------------------------------------------------------------- timeout self-test
+
+// One thread waits, through the kernels' bounded barrier wait, on a barrier
+// that nothing completes: after `limit` cycles the wait records
+// TPLA_ERR_DEVICE_TIMEOUT in the status word and returns, and the kernel
+// exits.  Lets a test exercise the timeout path without faulting the GPU.
+__global__ void wait_timeout_selftest_kernel(long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_addr(&bar);
+  mbar_init(b, 1);
+  abort_flag = 0;
+  fence_mbar_init();
+  wait_bar(b, 0, &abort_flag, limit);
+}
+
 // ---------------------------------------------------------------- host side
 
 struct DeviceInfo {
@@ -1215,6 +1233,12 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
     e = cudaGetLastError();
   }
   return e;
+}
+
+cudaError_t launch_wait_timeout_selftest(long long cycles, cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(cycles);
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t status_read_clear_sm100(int* code) {

@@ -83,5 +83,6 @@ void count_launch(int n = 1);
 // these read and clear it (after the caller synchronised the stream).
 cudaError_t status_read_clear_generic(int* code);
 cudaError_t status_read_clear_sm100(int* code);
+cudaError_t launch_wait_timeout_selftest(long long cycles, cudaStream_t stream);
 
 }  // namespace tpla

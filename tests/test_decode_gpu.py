@@ -157,6 +157,21 @@ def test_bad_page_id_sets_status(cuda_dev, kernel):
     assert_out_close(o[[0, 2]], ro)
 
 
+def test_device_wait_timeout_is_reported_and_context_survives(cuda_dev):
+    """A bounded barrier wait that nothing completes gives up after ~1 ms,
+    records TPLA_ERR_DEVICE_TIMEOUT and returns: no hang, no fault, and the
+    next decode on the same context is correct."""
+    assert tp.device_status() == 0
+    tp.selftest_wait_timeout(1000)
+    assert tp.device_status() == -5
+    assert tp.device_status() == 0  # cleared by the read
+    w = make_workload("tiny")
+    out, lse = run(cuda_dev, w, 1, "replicate", "sm100")
+    ro, rl = oracle_decode(w, 1, "replicate")
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+
+
 def test_hadamard_end_to_end_g1_invariance(cuda_dev):
     """Rotate q and cache on the GPU, decode exact MLA, un-rotate the output:
     equals the unrotated oracle (U U^T = I), through one bf16 re-rounding of
