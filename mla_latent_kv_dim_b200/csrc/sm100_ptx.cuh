@@ -32,12 +32,6 @@ __device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n"
                "barrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -61,20 +55,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-// Arrive on a barrier given by its shared::cluster address (any CTA).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
-               : "memory");
-}
-
-// Arrive on a barrier given by its shared::cluster address, with the default
-// (CTA-scope) release: the form 2-CTA tensor-core pipelines use to hand a
-// shared-memory operand to the peer's MMA after fence.proxy.async.  The
-// cluster-scope release above costs ~2000 cycles per arrival.
+// Arrive on a barrier given by its shared::cluster address (any CTA of the
+// cluster), with the default (CTA-scope) release: the form 2-CTA tensor-core
+// pipelines use to hand a shared-memory operand to the peer's MMA after
+// fence.proxy.async.  (A .release.cluster arrive costs ~2000 cycles.)
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
@@ -161,19 +145,8 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread for the CTA pair.
-__device__ __forceinline__ void mma_pair_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      :
-      : "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The same MMA with each descriptor given as 32-bit halves: the low half
+// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread for the CTA pair,
+// with each shared-memory descriptor given as 32-bit halves: the low half
 // (start address and leading offset) varies per operand, the high half is
 // constant per layout.  Fewer issuing instructions per MMA matter because
 // the issuing thread shares its SM sub-partition with busy softmax warps.
