@@ -41,6 +41,7 @@ from mla_latent_kv_dim_b200.workloads import (LATENT, ROPE, WIDTH, CONFIGS,  # n
 
 METRIC = "latent-KV GB/s & decode tok/s/layer at H=128 L=32K (% HBM peak), vs G"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (DGX figure); context beside the measured copy
 
 
 def parse_args():
@@ -81,6 +82,19 @@ def flops_per_token_head(G, shard=None, rope_mode="replicate"):
     r = ROPE if rope_mode == "replicate" else ROPE // G
     shards = G if shard is None else 1
     return shards * (2 * (d + r) + 2 * d)
+
+
+def one_shard_speedups(vs_G):
+    """Decode time of exact MLA (G=1, every latent column) over the time of
+    one TPLA shard's read (one-shard mode), per G: the per-rank attention
+    speedup that the pages' end-to-end TPLA-vs-MLA decode speedups at 32K
+    context stem from.  None without a G=1 entry."""
+    t = {(e["G"], e["mode"]): e["decode_us"] for e in vs_G}
+    base = t.get((1, "full"))
+    if not base:
+        return None
+    return {f"G{g}": round(base / t[(g, "one-shard")], 3)
+            for g in sorted({e["G"] for e in vs_G}) if (g, "one-shard") in t}
 
 
 def decode_kernel_hash():
@@ -493,6 +507,7 @@ def run_ours(args):
     roof.update({"traffic": traffic, "kernel": kname,
                  "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
                  "hbm_gbs": round(achieved_gbs, 1), "hbm_frac": round(achieved_gbs / hbm_peak, 4),
+                 "hbm_frac_nominal_8tbs": round(achieved_gbs / NOMINAL_HBM_GBS, 4),
                  "tensor_tflops": round(achieved_tf, 2),
                  "tensor_frac_burst": round(achieved_tf / tc_peak, 4),
                  "bytes_per_launch": bytes_step, "flops_per_launch": flops_step,
@@ -546,7 +561,8 @@ def run_ours(args):
         "config": step_config(args, w, used, f"replicas x{world}"),
         "tok_s_layer": round(tok_s, 1),
         "hbm_frac_step": round(value / world / hbm_peak, 4),
-        "roofline": roof, "vs_G": vs_G, "cpu_baseline": cpu,
+        "roofline": roof, "vs_G": vs_G, "one_shard_speedup_vs_mla": one_shard_speedups(vs_G),
+        "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "pipelining": "H2D, compute and D2H on three streams, two buffer sets",
                 "serial_value": round(e2e_serial, 2),

@@ -48,3 +48,13 @@ def test_benchmark_arithmetic_intensity():
     # the DeepSeek-V3 step (G=2, rope replicated): 2304 flops per token-head,
     # 1152 bytes per token, 128 heads -> 256 flops per byte
     assert bench.flops_per_token_head(2) * 128 / 1152 == 256
+
+
+def test_one_shard_speedups_divide_g1_time_by_the_shard_time():
+    vs_G = [{"G": 1, "mode": "full", "decode_us": 800.0},
+            {"G": 2, "mode": "full", "decode_us": 810.0},
+            {"G": 2, "mode": "one-shard", "decode_us": 400.0},
+            {"G": 4, "mode": "one-shard", "decode_us": 320.0}]
+    assert bench.one_shard_speedups(vs_G) == {"G2": 2.0, "G4": 2.5}
+    assert bench.one_shard_speedups([]) is None
+    assert bench.one_shard_speedups(vs_G[1:]) is None
