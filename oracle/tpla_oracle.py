@@ -40,6 +40,18 @@ Readings taken where the pages are silent:
    output 0 and lse = -inf.
 7. The Hadamard transform is the orthonormal Sylvester (natural-order) matrix
    applied to the first ``dim`` columns of a row.
+8. PCA is taken over the calibration rows' latent columns only (position
+   features excluded): the covariance of the mean-centred rows,
+   (1/N) sum (f - m)^T (f - m).  U holds the unit eigenvectors as columns in
+   descending eigenvalue order, each signed so that its entry of largest
+   magnitude (the first such, on a tie) is positive.  Only the rotation
+   x -> x U is applied to q and the cache; the mean is not subtracted.
+9. Eq. (25)'s alpha and beta are the shares of the eigenvalue sum in shard
+   0's and shard 1's index ranges, taken disjoint ([0, d) and [d, 2d)), which
+   fixes the overlap at lambda_{d/2} the referee points out; for G shards
+   each shard's share is taken the same way.  They are diagnostics: the
+   deployed computation is the unscaled local softmax (reading 1), so no
+   mu/nu factor enters it.
 """
 
 from __future__ import annotations
@@ -339,6 +351,72 @@ def hadamard_ref(x, dim):
     Hm = hadamard_matrix(dim)
     x[..., :dim] = x[..., :dim] @ Hm  # H is symmetric: row-vector form
     return x
+
+
+# ---------------------------------------------------------------------------
+# PCA reparameterisation (the pages' other orthogonal transform)
+# ---------------------------------------------------------------------------
+
+def pca_basis_ref(F):
+    """Principal axes of calibration latents ``F`` [N, D] (reading 8).
+
+    [ABSTRACT] and [ISSUE] "Directions under investigation": an orthogonal
+    transform such as PCA is applied before TP slicing.  [REVIEW referee
+    report, minor comment on Sec. 4.3.2 / Eq. (25)]: PCA of the collected
+    latent features, position features excluded.  [REVIEW pith extraction,
+    key machinery]: the orthogonal U is absorbed into the MLA projections.
+    The symmetric eigensolver is a library primitive.  Returns
+    (lam [D] descending, U [D, D] with the eigenvectors as columns).
+    """
+    F = np.asarray(F, np.float64)
+    if F.ndim != 2 or F.shape[0] == 0:
+        raise ValueError("F must be [N, D] with N > 0")
+    Fc = F - F.mean(axis=0, keepdims=True)
+    C = Fc.T @ Fc / F.shape[0]
+    lam, V = np.linalg.eigh(C)
+    order = np.argsort(-lam, kind="stable")
+    lam, V = lam[order], V[:, order]
+    lead = np.argmax(np.abs(V), axis=0)
+    sign = np.sign(V[lead, np.arange(V.shape[1])])
+    return lam, V * np.where(sign == 0, 1.0, sign)
+
+
+def pca_calibrate_ref(rows):
+    """PCA basis from calibration cache rows [N, 576]: latent columns only,
+    the rope part excluded (reading 8)."""
+    rows = np.asarray(rows, np.float64)
+    return pca_basis_ref(rows[:, :LATENT])
+
+
+def shard_variance_fractions(lam, G):
+    """Each shard's share of the eigenvalue sum over its contiguous index
+    range [g d, (g + 1) d), d = len(lam) / G; for G = 2 these are Eq. (25)'s
+    alpha and beta with disjoint ranges (reading 9)."""
+    lam = np.asarray(lam, np.float64)
+    if lam.shape[0] % G:
+        raise ValueError("G must divide the dimension")
+    d = lam.shape[0] // G
+    return np.array([lam[g * d:(g + 1) * d].sum() for g in range(G)]) / lam.sum()
+
+
+def pca_rotate_ref(x, U, dim=LATENT):
+    """x[..., :dim] <- x[..., :dim] U on every row; other columns (rope)
+    unchanged.  The same U rotates q's latent part and the cache rows, so the
+    global latent logits q c^T are unchanged (U U^T = I)."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    x[..., :dim] = x[..., :dim] @ np.asarray(U, np.float64)
+    return x
+
+
+def pca_unrotate_ref(out_latent, U):
+    """Back from the rotated latent space: out U^T."""
+    return np.asarray(out_latent, np.float64) @ np.asarray(U, np.float64).T
+
+
+def fold_vup_ref(W_uv, U):
+    """V-up weights for outputs in the rotated space: W'[h] = U^T W[h], so
+    that (out U) W' = out W (the rotation absorbed into the projection)."""
+    return np.einsum("ji,hjk->hik", np.asarray(U, np.float64), np.asarray(W_uv, np.float64))
 
 
 # ---------------------------------------------------------------------------

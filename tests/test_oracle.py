@@ -301,6 +301,156 @@ def test_hadamard_changes_tpla_g2():
     assert not np.allclose(o, O.hadamard_ref(o2, 512), atol=1e-6)
 
 
+# ---------------------------------------------------------------- PCA
+
+def _design(N, D):
+    """N x D of +-1 whose columns are zero-mean and mutually orthogonal
+    (Z^T Z = N I): non-constant Walsh columns from scipy's Hadamard."""
+    from scipy.linalg import hadamard
+    return hadamard(N).astype(np.float64)[:, 1:D + 1]
+
+
+def _planted(offset=1.5):
+    """Calibration rows with a known covariance R diag(s^2) R^T (plus a
+    constant offset that centring must remove), and the basis the pages'
+    PCA must return: R's columns by descending s^2.  R is four plane
+    rotations by angles below 45 degrees, so each column's largest entry is
+    already positive."""
+    D = 8
+    R = np.zeros((D, D))
+    for k, th in enumerate([0.3, 0.5, 0.1, 0.7]):
+        c, s_ = math.cos(th), math.sin(th)
+        R[2 * k:2 * k + 2, 2 * k:2 * k + 2] = [[c, -s_], [s_, c]]
+    var = np.array([5.0, 0.5, 3.0, 7.0, 1.0, 2.0, 9.0, 4.0])
+    F = (_design(64, D) * np.sqrt(var)) @ R.T + offset
+    order = [6, 3, 0, 7, 2, 5, 4, 1]
+    return F, var[order], R[:, order]
+
+
+def _matches_planted(basis_fn):
+    F, lam_x, U_x = _planted()
+    lam, U = basis_fn(F)
+    return np.allclose(lam, lam_x, atol=1e-12) and np.allclose(U, U_x, atol=1e-12)
+
+
+def test_pca_recovers_planted_eigenpairs():
+    assert _matches_planted(O.pca_basis_ref)
+    F, _, _ = _planted()
+    lam, U = O.pca_basis_ref(F)
+    assert np.allclose(U.T @ U, np.eye(8), atol=1e-13)
+
+
+def test_pca_sign_rule_on_a_tie():
+    """45-degree axes: entries tie in magnitude, so the first is made
+    positive: (1, 1)/sqrt2 for the larger variance, (1, -1)/sqrt2 next."""
+    Z = _design(16, 2)
+    F = (Z * [2.0, 1.0]) @ (np.array([[1.0, -1.0], [1.0, 1.0]]) / math.sqrt(2)).T
+    lam, U = O.pca_basis_ref(F)
+    assert np.allclose(lam, [4.0, 1.0], atol=1e-13)
+    assert np.allclose(U, np.array([[1.0, 1.0], [1.0, -1.0]]) / math.sqrt(2), atol=1e-13)
+
+
+def test_pca_fractions_of_the_decayed_cache_closed_form():
+    """Uncorrelated latent channels with standard deviation exp(-j/128), the
+    workloads' decay, stored in a scrambled channel order: PCA sorts them
+    back (U is the inverse permutation), lam_j = exp(-j/64), and shard g of G
+    holds r^(g d) (1 - r^d) / (1 - r^512) of the sum, r = exp(-1/64); at G = 2
+    alpha = 1 / (1 + e^-4) and alpha + beta = 1."""
+    D = 512
+    s = np.exp(-np.arange(D) / 128.0)
+    perm = np.random.default_rng(3).permutation(D)
+    F = (_design(1024, D) * s)[:, perm]
+    lam, U = O.pca_basis_ref(F)
+    assert np.allclose(lam, s ** 2, rtol=1e-10, atol=0)
+    assert np.allclose(U, np.eye(D)[:, np.argsort(perm)], atol=1e-10)
+    a, b = O.shard_variance_fractions(lam, 2)
+    assert abs(a - 1.0 / (1.0 + math.exp(-4.0))) < 1e-12
+    assert abs(a + b - 1.0) < 1e-14
+    r = math.exp(-1.0 / 64.0)
+    for G in (4, 8):
+        d = D // G
+        want = [r ** (g * d) * (1 - r ** d) / (1 - r ** D) for g in range(G)]
+        assert np.allclose(O.shard_variance_fractions(lam, G), want, rtol=1e-10, atol=0)
+
+
+def test_pca_isotropic_shares_are_equal():
+    lam, _ = O.pca_basis_ref(_design(64, 16) * 3.0)
+    assert np.allclose(lam, 9.0, atol=1e-12)
+    for G in (1, 2, 4, 8):
+        assert np.allclose(O.shard_variance_fractions(lam, G), 1.0 / G, atol=1e-14)
+
+
+def test_pca_leading_axis_matches_power_iteration():
+    """Power iteration on the centred rows, an algorithm independent of the
+    library eigensolver, finds the same leading axis and eigenvalue."""
+    rng = np.random.default_rng(11)
+    N, D = 400, 16
+    F = rng.standard_normal((N, D)) @ np.diag(np.linspace(3.0, 0.5, D)) + 2.0
+    lam, U = O.pca_basis_ref(F)
+    Fc = F - F.mean(axis=0)
+    v = np.ones(D)
+    for _ in range(3000):
+        v = Fc.T @ (Fc @ v)
+        v /= np.linalg.norm(v)
+    v = v if v[np.argmax(np.abs(v))] > 0 else -v
+    assert np.allclose(U[:, 0], v, atol=1e-8)
+    assert abs(lam[0] - v @ (Fc.T @ (Fc @ v)) / N) < 1e-10
+
+
+def test_pca_calibration_excludes_rope():
+    """The basis comes from the latent columns alone: rope columns with a
+    large, correlated variance change nothing."""
+    rng = np.random.default_rng(17)
+    lat = rng.standard_normal((300, 512)) * np.exp(-np.arange(512) / 128.0)
+    rope = 50.0 * lat[:, :64] + rng.standard_normal((300, 64))
+    lam, U = O.pca_calibrate_ref(np.concatenate([lat, rope], axis=1))
+    lam2, U2 = O.pca_basis_ref(lat)
+    assert U.shape == (512, 512)
+    assert np.array_equal(lam, lam2) and np.array_equal(U, U2)
+
+
+def test_pca_rotation_invariance_for_g1_and_fold():
+    """U absorbed into q and the cache leaves exact MLA unchanged after the
+    output is rotated back, and folding U^T into W_uv gives the same y."""
+    rng = np.random.default_rng(19)
+    _, U = O.pca_basis_ref(rng.standard_normal((700, 512)) * np.exp(-np.arange(512) / 128.0))
+    q = _rand((2, 3, O.WIDTH), 181)
+    rows = _rows(2, [40, 65], 182)
+    o, l = O.tpla_decode_ref(q, rows, 1, "replicate", SCALE)
+    qr = O.pca_rotate_ref(q, U)
+    rr = [O.pca_rotate_ref(r, U) for r in rows]
+    assert np.array_equal(qr[..., 512:], q[..., 512:])
+    o2, l2 = O.tpla_decode_ref(qr, rr, 1, "replicate", SCALE)
+    assert np.allclose(O.pca_unrotate_ref(o2, U), o, atol=1e-12)
+    assert np.allclose(l2, l, atol=1e-12)
+    W = _rand((3, 512, 16), 183)
+    assert np.allclose(O.vup_ref(o2, O.fold_vup_ref(W, U)), O.vup_ref(o, W), atol=1e-10)
+    # for G = 2 the rotation is not absorbed exactly (shard-local softmax)
+    o3, _ = O.tpla_decode_ref(qr, rr, 2, "replicate", SCALE)
+    o4, _ = O.tpla_decode_ref(q, rows, 2, "replicate", SCALE)
+    assert not np.allclose(O.pca_unrotate_ref(o3, U), o4, atol=1e-6)
+
+
+def test_pca_pins_catch_planted_mistakes():
+    def ascending(F):
+        lam, U = O.pca_basis_ref(F)
+        return lam[::-1], U[:, ::-1]
+
+    def uncentred(F):
+        F = np.asarray(F, np.float64)
+        lam, V = np.linalg.eigh(F.T @ F / F.shape[0])
+        o = np.argsort(-lam)
+        V = V[:, o]
+        return lam[o], V * np.sign(V[np.argmax(np.abs(V), axis=0), np.arange(V.shape[1])])
+
+    def transposed(F):
+        lam, U = O.pca_basis_ref(F)
+        return lam, U.T
+
+    for bad in (ascending, uncentred, transposed):
+        assert not _matches_planted(bad)
+
+
 # ---------------------------------------------------------------- combine
 
 @pytest.mark.parametrize("G", [1, 2, 4])
