@@ -144,7 +144,10 @@ TPLA_API int tpla_decode_ex(const tpla_tensor* q, const tpla_tensor* kv_cache,
 /*
  * tpla_decode_workspace_size -- bytes of device workspace tpla_decode_ex
  * needs for these arguments and options (0 when no split is used).  Same
- * validation as tpla_decode_ex; writes the size to *bytes.
+ * validation as tpla_decode_ex; writes the size to *bytes.  With
+ * TPLA_KERNEL_AUTO the size covers either kernel, because the automatic
+ * choice also depends on the scale, which this query does not take (a
+ * scale <= 0 runs the generic kernel).
  */
 TPLA_API int tpla_decode_workspace_size(const tpla_tensor* q, const tpla_tensor* kv_cache,
                                const tpla_tensor* seq_lens,

@@ -200,7 +200,18 @@ int tpla_decode_workspace_size(const tpla_tensor* q, const tpla_tensor* kv_cache
   Path path;
   rc = choose_path(p, opts, &path);
   if (rc != TPLA_OK) return rc;
-  return workspace_needed(p, opts, path, bytes);
+  rc = workspace_needed(p, opts, path, bytes);
+  if (rc != TPLA_OK) return rc;
+  // The automatic choice also depends on the scale, which this query does not
+  // take (a scale <= 0 runs the generic kernel), so size for either kernel.
+  const int choice = opts ? opts->kernel : TPLA_KERNEL_AUTO;
+  if (choice == TPLA_KERNEL_AUTO && path == Path::Sm100) {
+    size_t g = 0;
+    rc = workspace_needed(p, opts, Path::Generic, &g);
+    if (rc != TPLA_OK) return rc;
+    if (g > *bytes) *bytes = g;
+  }
+  return TPLA_OK;
 }
 
 int tpla_decode_ex(const tpla_tensor* q, const tpla_tensor* kv_cache,
