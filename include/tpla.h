@@ -134,6 +134,10 @@ typedef struct {
  * Kernel choice (opts->kernel = AUTO): the tcgen05 kernel when the device is
  * sm_100, G is 1, 2 or 4, H <= 128, scale > 0 and out rows are 16-byte
  * aligned; the portable kernel otherwise.  Both compute the same function.
+ *
+ * Size limits (TPLA_ERR_UNSUPPORTED beyond them, nothing launched):
+ * B <= 2^20, H <= 4096, B * H <= 2^30, num_splits <= 65535,
+ * B * num_splits <= 2^24, and on the portable kernel B * shards <= 65535.
  */
 TPLA_API int tpla_decode_ex(const tpla_tensor* q, const tpla_tensor* kv_cache,
                    const tpla_tensor* seq_lens, const tpla_tensor* page_table,
@@ -206,6 +210,7 @@ TPLA_API int tpla_decode_noalloc(const tpla_tensor* q, const tpla_tensor* kv_cac
  *   out       [B, H, Wd] f32 or bf16;  lse NULL or [B, H, Gs] f32.
  * lse = ln sum_s exp(lse_s); out = sum_s exp(lse_s - lse) o_s.  Chunks with
  * lse = -inf contribute nothing; if every chunk is -inf, out = 0, lse = -inf.
+ * Limits (TPLA_ERR_UNSUPPORTED): S <= 1024, B * H <= 2^30, Wd <= 2^20.
  */
 TPLA_API int tpla_lse_merge(const tpla_tensor* o_parts, const tpla_tensor* lse_parts,
                    tpla_tensor* out, tpla_tensor* lse, tpla_stream_t stream);

@@ -21,6 +21,12 @@ int cuda_fail(cudaError_t e) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Launch-geometry limits the entry points check before any launch.
+constexpr int kMaxSplits = 65535;                     // a grid dimension of the generic kernel
+constexpr int64_t kMaxRequestHeads = 1LL << 30;       // B * H: merge blocks, 32-bit grid
+constexpr int64_t kMaxRequestSplits = 1LL << 24;      // B * num_splits: 2x that many slots
+constexpr int64_t kMaxGenericRequestShards = 65535;   // B * shards: the generic grid's z
+
 bool check_tensor(const tpla_tensor* t, int dtype, int ndim) {
   if (!t || t->dtype != dtype || t->ndim != ndim) return false;
   for (int i = 0; i < ndim; ++i) {
@@ -52,12 +58,17 @@ int build_problem(const tpla_tensor* q, const tpla_tensor* kv, const tpla_tensor
   int shard = opts ? opts->shard : -1;
   if (shard < -1 || shard >= G) return TPLA_ERR_INVALID_ARG;
   if (opts && (opts->reserved != 0 || opts->num_splits < 0)) return TPLA_ERR_INVALID_ARG;
+  if (opts && opts->num_splits > kMaxSplits) return TPLA_ERR_UNSUPPORTED;
   if (opts && (opts->kernel < TPLA_KERNEL_AUTO || opts->kernel > TPLA_KERNEL_SM100))
     return TPLA_ERR_INVALID_ARG;
 
   if (!check_tensor(q, TPLA_BF16, 3) || q->shape[2] != kWidth) return TPLA_ERR_INVALID_ARG;
   const int64_t B = q->shape[0], H = q->shape[1];
   if (B > (1 << 20) || H > 4096) return TPLA_ERR_UNSUPPORTED;
+  // (request, head) pairs index one merge block each; explicit splits index
+  // 2 * B * num_splits partial slots
+  if (B * H > kMaxRequestHeads) return TPLA_ERR_UNSUPPORTED;
+  if (opts && B * opts->num_splits > kMaxRequestSplits) return TPLA_ERR_UNSUPPORTED;
   if (!check_tensor(seq, TPLA_I32, 1) || seq->shape[0] != B) return TPLA_ERR_INVALID_ARG;
   if (!check_tensor(kv, TPLA_BF16, 3) || kv->shape[2] != kWidth) return TPLA_ERR_INVALID_ARG;
   const bool paged = pt != nullptr;
@@ -140,6 +151,8 @@ int choose_path(const DecodeProblem& p, const tpla_decode_opts* opts, Path* path
   } else {
     *path = fast ? Path::Sm100 : Path::Generic;
   }
+  if (*path == Path::Generic && (int64_t)p.B * p.n_shards > kMaxGenericRequestShards)
+    return TPLA_ERR_UNSUPPORTED;
   return TPLA_OK;
 }
 
@@ -271,7 +284,7 @@ int tpla_lse_merge(const tpla_tensor* o_parts, const tpla_tensor* lse_parts, tpl
   if (lse_parts->shape[0] != S || lse_parts->shape[1] != B || lse_parts->shape[2] != H)
     return TPLA_ERR_INVALID_ARG;
   if (Gs < 1 || Wd % Gs != 0 || S < 1) return TPLA_ERR_INVALID_ARG;
-  if (S > 1024) return TPLA_ERR_UNSUPPORTED;
+  if (S > 1024 || B * H > kMaxRequestHeads || Wd > (1 << 20)) return TPLA_ERR_UNSUPPORTED;
   if (!out || (out->dtype != TPLA_F32 && out->dtype != TPLA_BF16) ||
       !check_tensor(out, out->dtype, 3) || out->shape[0] != B || out->shape[1] != H ||
       out->shape[2] != Wd)

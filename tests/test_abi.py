@@ -119,6 +119,48 @@ def test_validation_rejects_without_launch(mutate):
     assert tp.launch_count() == 0
 
 
+@pytest.mark.parametrize("case", ["splits", "request_heads", "request_splits",
+                                  "generic_grid"])
+def test_size_limits_are_unsupported_without_launch(case):
+    """Sizes whose launch geometry the kernels cannot express come back as
+    TPLA_ERR_UNSUPPORTED before anything is launched."""
+    before = tp.launch_count()
+    G, opts = 2, None
+    if case == "splits":
+        q, kv, seq, pt, out, lse = _good()
+        opts = N._opts(65536, None, "auto")
+    elif case == "request_heads":  # B * H > 2^30
+        q, kv, seq, pt, out, lse = _good(B=1 << 20, H=2048)
+    elif case == "request_splits":  # B * num_splits > 2^24
+        q, kv, seq, pt, out, lse = _good(B=1 << 12)
+        opts = N._opts(1 << 13, None, "auto")
+    else:  # the portable kernel's grid: B * shards > 65535
+        G = 8
+        q, kv, seq, pt, out, lse = _good(B=10000, G=8)
+        opts = N._opts(0, None, "generic")
+    assert _call(q, kv, seq, pt, G, 0, out, lse, opts) == -2
+    n = ctypes.c_size_t(0)
+    rc = tp.lib().tpla_decode_workspace_size(ctypes.byref(q), ctypes.byref(kv), ctypes.byref(seq),
+                                             ctypes.byref(pt), G, 0, ctypes.byref(out),
+                                             ctypes.byref(opts) if opts else None,
+                                             ctypes.byref(n))
+    assert rc == -2
+    assert tp.launch_count() == before
+
+
+def test_lse_merge_size_limits():
+    o = _fake((2, 1 << 16, 1 << 15, 8), torch.float32)
+    lp = _fake((2, 1 << 16, 1 << 15, 1), torch.float32)
+    out = _fake((1 << 16, 1 << 15, 8), torch.float32)
+    assert tp.lib().tpla_lse_merge(ctypes.byref(o), ctypes.byref(lp), ctypes.byref(out), None,
+                                   None) == -2
+    o = _fake((1025, 1, 1, 8), torch.float32)
+    lp = _fake((1025, 1, 1, 1), torch.float32)
+    out = _fake((1, 1, 8), torch.float32)
+    assert tp.lib().tpla_lse_merge(ctypes.byref(o), ctypes.byref(lp), ctypes.byref(out), None,
+                                   None) == -2
+
+
 def test_one_shard_shapes_validate():
     q, kv, seq, pt, out, lse = _good(G=4, shard=1)
     opts = N._opts(0, 1, "generic")
