@@ -116,6 +116,25 @@ def _ref(d):
     return ctypes.byref(d) if d is not None else None
 
 
+def _on_current_device(*tensors) -> None:
+    """libtpla receives raw device addresses and launches on the current
+    device, so every tensor must be a CUDA tensor on that device: a host
+    tensor or one on another GPU would be read at a wrong address."""
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"libtpla takes CUDA tensors; got one on {t.device}")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on different devices: {dev} and {t.device}")
+    if dev is not None and dev.index is not None and dev.index != torch.cuda.current_device():
+        raise ValueError(f"tensors are on {dev} but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
+
+
 def _stream(stream) -> int | None:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -137,6 +156,7 @@ def _opts(num_splits, shard, kernel, ws=None, ws_bytes=0) -> TplaDecodeOpts:
 
 def decode_workspace_size(q, kv_cache, seq_lens, page_table, G, rope_mode, out, *,
                           num_splits=0, shard=None, kernel="auto") -> int:
+    _on_current_device(q, kv_cache, seq_lens, page_table, out)
     n = ctypes.c_size_t(0)
     o = _opts(num_splits, shard, kernel)
     rc = lib().tpla_decode_workspace_size(
@@ -155,6 +175,7 @@ def decode(q, kv_cache, seq_lens, page_table, G=1, rope_mode="replicate", scale=
     """
     if scale is None:
         raise ValueError("scale is required")
+    _on_current_device(q, kv_cache, seq_lens, page_table, out, lse, workspace)
     B, H = q.shape[0], q.shape[1]
     width = 512 if shard is None else 512 // G
     n_sh = G if shard is None else 1
@@ -179,6 +200,7 @@ def decode(q, kv_cache, seq_lens, page_table, G=1, rope_mode="replicate", scale=
 def decode_simple(q, kv_cache, seq_lens, page_table, G, rope_mode, scale, out, lse=None,
                   stream=None):
     """``tpla_decode`` (default options, library-managed workspace)."""
+    _on_current_device(q, kv_cache, seq_lens, page_table, out, lse)
     rc = lib().tpla_decode(
         _ref(desc(q)), _ref(desc(kv_cache)), _ref(desc(seq_lens)), _ref(desc(page_table)),
         int(G), ROPE_MODES[rope_mode], ctypes.c_float(scale), _ref(desc(out)), _ref(desc(lse)),
@@ -188,6 +210,7 @@ def decode_simple(q, kv_cache, seq_lens, page_table, G, rope_mode, scale, out, l
 
 
 def lse_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
+    _on_current_device(o_parts, lse_parts, out, lse)
     S, B, H, Wd = o_parts.shape
     if out is None:
         out = torch.empty((B, H, Wd), dtype=torch.float32, device=o_parts.device)
@@ -201,12 +224,14 @@ def lse_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
 
 def hadamard_apply(buf, dim=512, stream=None):
     """In-place orthonormal Walsh-Hadamard transform of buf[..., :dim]."""
+    _on_current_device(buf)
     rc = lib().tpla_hadamard_apply(_ref(desc(buf)), int(dim), _stream(stream))
     _check("tpla_hadamard_apply", rc)
     return buf
 
 
 def vup_combine(out_latent, W_uv, y=None, stream=None):
+    _on_current_device(out_latent, W_uv, y)
     B, H = out_latent.shape[0], out_latent.shape[1]
     if y is None:
         y = torch.empty((B, H, W_uv.shape[2]), dtype=torch.float32, device=out_latent.device)

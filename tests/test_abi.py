@@ -210,3 +210,38 @@ def test_hadamard_and_vup_validation():
     y = _fake((2, 4, 128), torch.float32)
     assert L.tpla_vup_combine(ctypes.byref(o), ctypes.byref(W), ctypes.byref(y), None) == -1
     assert tp.launch_count() == 0
+
+
+def test_binding_rejects_host_tensors_before_the_library():
+    """The binding hands raw addresses to kernels, so host tensors are refused
+    in Python before any library call."""
+    before = tp.launch_count()
+    q = torch.zeros((1, 16, 576), dtype=torch.bfloat16)
+    cache = torch.zeros((1, 64, 576), dtype=torch.bfloat16)
+    seq = torch.ones((1,), dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        tp.decode(q, cache, seq, None, 1, "replicate", 0.07)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        tp.hadamard_apply(torch.zeros((4, 512)), 512)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        tp.vup_combine(torch.zeros((1, 1, 512)), torch.zeros((1, 512, 128), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        tp.lse_merge(torch.zeros((2, 1, 1, 8)), torch.zeros((2, 1, 1, 1)))
+    assert tp.launch_count() == before
+
+
+class _OnCuda:
+    """Stands in for a CUDA tensor: only what the device check reads."""
+    is_cuda = True
+
+    def __init__(self, index):
+        self.device = torch.device("cuda", index)
+
+
+def test_binding_device_check(monkeypatch):
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    N._on_current_device(_OnCuda(0), None, _OnCuda(0))
+    with pytest.raises(ValueError, match="different devices"):
+        N._on_current_device(_OnCuda(0), _OnCuda(1))
+    with pytest.raises(ValueError, match="current device"):
+        N._on_current_device(_OnCuda(1), _OnCuda(1))
