@@ -245,3 +245,13 @@ def test_binding_device_check(monkeypatch):
         N._on_current_device(_OnCuda(0), _OnCuda(1))
     with pytest.raises(ValueError, match="current device"):
         N._on_current_device(_OnCuda(1), _OnCuda(1))
+
+
+@pytest.mark.parametrize("B,H", [(0, 16), (2, 0)])
+def test_empty_batch_or_heads_is_a_no_op(B, H):
+    """No requests (or no heads) is a valid call that launches nothing."""
+    before = tp.launch_count()
+    q, kv, seq, pt, out, lse = _good(B=B, H=H)
+    assert _call(q, kv, seq, pt, 2, 0, out, lse) == 0
+    assert _call(q, kv, seq, pt, 2, 0, out, lse, N._opts(0, None, "generic")) == 0
+    assert tp.launch_count() == before
