@@ -1,9 +1,10 @@
 // Log-sum-exp merge of split-KV partial results.
 //
-// The exact sequence-split alternative of the feature request "Bandwidth-
-// optimal tensor-parallel sharding of MLA" (section "Directions under
-// investigation": sequence split + flash-attention log-sum-exp merge):
-// chunk s of a request produced a normalised output o_s and lse_s, then
+// The exact alternative of the feature request "Bandwidth-optimal
+// tensor-parallel sharding of MLA" (section "Directions under
+// investigation") that splits the sequence and combines the pieces by their
+// log-sum-exp: chunk s of a request produced a normalised output o_s and
+// lse_s, then
 //   lse = M + ln sum_s exp(lse_s - M),  M = max_s lse_s
 //   out = sum_s exp(lse_s - lse) o_s.
 // Empty chunks carry lse = -inf and weigh nothing; a request whose chunks

@@ -73,8 +73,9 @@ BLOCK = 64    # tokens per cache page
 def shard_columns(G: int, g: int, rope_mode: str = "replicate"):
     """Return (latent_cols, rope_cols) of shard ``g`` out of ``G``.
 
-    [ABSTRACT]: TPLA partitions the latent representation and each head's
-    input dimension across devices.  [REVIEW referee_report.significance]:
+    [ABSTRACT]: the latent vector, and with it the matching slice of every
+    head's query, is cut into per-device pieces.  [REVIEW
+    referee_report.significance]:
     the per-device cache is 256 + 64 = 320 dims at TP=2, so the rope part is
     replicated to every shard.  ``split`` (rope also cut into G slices) is
     the alternative reading; contiguous slices in shard order (readings 2, 3).
@@ -197,10 +198,12 @@ def mla_decode_ref(q, rows, scale):
 def tpla_decode_ref(q, rows, G, rope_mode, scale, shard=None):
     """TPLA decode: G latent shards, an independent softmax per shard.
 
-    [ISSUE] "Directions under investigation": each rank runs local attention
-    over its latent slice.  [REVIEW pith_extraction.key_machinery]: device i
-    computes softmax(Q_i (cKV_i U)^T) with all query heads replicated;
-    [REVIEW skeptic_critique]: Eq. 6 is an unscaled local softmax.
+    [ISSUE] "Directions under investigation": every rank attends only over
+    the latent columns it holds.  [REVIEW pith_extraction.key_machinery]:
+    on each device the softmax is taken over the product of every head's
+    query slice with that device's rotated cache slice;
+    [REVIEW skeptic_critique]: Eq. 6 applies no scaling to that local
+    softmax.
     Shard g's logits use its latent columns plus its rope columns; its
     values are its latent columns only.  Outputs are concatenated in shard
     order (reading 5).

@@ -102,7 +102,7 @@ def test_mla_matches_bruteforce():
 # ---------------------------------------------------------------- invariants
 
 def test_g1_equals_exact_mla():
-    """'G=1 matches head-TP MLA exactly' (issue, Tests / validation)."""
+    """With one shard TPLA is exact MLA (issue, Tests / validation)."""
     B, H = 3, 4
     q = _rand((B, H, O.WIDTH), 31)
     rows = _rows(B, [9, 1, 33], 32)
