@@ -360,6 +360,17 @@ def hadamard_ref(x, dim):
 # PCA reparameterisation (the pages' other orthogonal transform)
 # ---------------------------------------------------------------------------
 
+def latent_covariance_ref(F):
+    """Mean [D] and covariance [D, D] of calibration rows ``F`` [N, D]: the
+    mean-centred second moment (1/N) sum (f - m)^T (f - m) (reading 8)."""
+    F = np.asarray(F, np.float64)
+    if F.ndim != 2 or F.shape[0] == 0:
+        raise ValueError("F must be [N, D] with N > 0")
+    m = F.mean(axis=0)
+    Fc = F - m
+    return m, Fc.T @ Fc / F.shape[0]
+
+
 def pca_basis_ref(F):
     """Principal axes of calibration latents ``F`` [N, D] (reading 8).
 
@@ -371,11 +382,7 @@ def pca_basis_ref(F):
     The symmetric eigensolver is a library primitive.  Returns
     (lam [D] descending, U [D, D] with the eigenvectors as columns).
     """
-    F = np.asarray(F, np.float64)
-    if F.ndim != 2 or F.shape[0] == 0:
-        raise ValueError("F must be [N, D] with N > 0")
-    Fc = F - F.mean(axis=0, keepdims=True)
-    C = Fc.T @ Fc / F.shape[0]
+    _, C = latent_covariance_ref(F)
     lam, V = np.linalg.eigh(C)
     order = np.argsort(-lam, kind="stable")
     lam, V = lam[order], V[:, order]

@@ -340,6 +340,16 @@ def test_pca_recovers_planted_eigenpairs():
     assert np.allclose(U.T @ U, np.eye(8), atol=1e-13)
 
 
+def test_covariance_of_planted_rows():
+    """The planted rows' mean is the offset and their covariance is
+    R diag(var) R^T, whatever the offset."""
+    for off in (0.0, 1.5, -40.0):
+        F, lam_x, U_x = _planted(off)
+        m, C = O.latent_covariance_ref(F)
+        assert np.allclose(m, off, atol=1e-12)
+        assert np.allclose(C, U_x @ np.diag(lam_x) @ U_x.T, atol=1e-11)
+
+
 def test_pca_sign_rule_on_a_tie():
     """45-degree axes: entries tie in magnitude, so the first is made
     positive: (1, 1)/sqrt2 for the larger variance, (1, -1)/sqrt2 next."""
