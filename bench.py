@@ -227,13 +227,14 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_sample(w, G, rope, hadamard, budget_s):
+def oracle_sample(w, G, rope, hadamard, budget_s, prepared=None):
     """Time the float64 oracle on whole requests of the workload, doing what
     one GPU step does per request: decode (on the stored, already rotated
     cache when the Hadamard is folded in) and the V-up combine.  The rotation
     itself is set-up on both sides and is not timed.  Runs until about
-    ``budget_s`` seconds of oracle time have passed.  Returns (GB/s, seconds,
-    requests)."""
+    ``budget_s`` seconds of oracle time have passed.  ``prepared`` (a dict)
+    keeps each request's gathered, rotated rows between calls, as the stored
+    cache stays between GPU steps.  Returns (GB/s, seconds, requests)."""
     from oracle import tpla_oracle as O  # CPU baseline leg only
     from mla_latent_kv_dim_b200.workloads import as_f64
     Wv = as_f64(w.W_uv) if w.W_uv is not None else None
@@ -245,15 +246,21 @@ def oracle_sample(w, G, rope, hadamard, budget_s):
     b = 0
     while t_total < budget_s and b < w.B:
         L = int(w.seq_lens[b])
-        pages = (L + 63) // 64
-        if w.page_table is not None:
-            rows = as_f64(w.cache[w.page_table[b, :pages].long()].reshape(pages * 64, WIDTH)[:L])
+        if prepared is not None and b in prepared:
+            q, rows = prepared[b]
         else:
-            rows = as_f64(w.cache[b, :L])
-        q = as_f64(w.q[b:b + 1])
-        if hadamard:
-            q = O.hadamard_ref(q, 512)
-            rows = O.hadamard_ref(rows, 512)
+            pages = (L + 63) // 64
+            if w.page_table is not None:
+                rows = as_f64(w.cache[w.page_table[b, :pages].long()].reshape(pages * 64,
+                                                                              WIDTH)[:L])
+            else:
+                rows = as_f64(w.cache[b, :L])
+            q = as_f64(w.q[b:b + 1])
+            if hadamard:
+                q = O.hadamard_ref(q, 512)
+                rows = O.hadamard_ref(rows, 512)
+            if prepared is not None:
+                prepared[b] = (q, rows)
         t0 = time.perf_counter()
         out, _ = O.tpla_decode_ref(q, [rows], G, rope, np.float32(w.scale))
         if Wv is not None:
@@ -289,9 +296,11 @@ def run_reference(args):
     hadamard = not args.no_hadamard
     per_step = []
     reqs = 0
+    prepared = {}
     for i in range(args.warmup + args.steps):
         gbs, t, n = oracle_sample(w, args.G, args.rope, hadamard,
-                                  budget_s=max(0.5, 120.0 / (args.warmup + args.steps)))
+                                  budget_s=max(0.5, 120.0 / (args.warmup + args.steps)),
+                                  prepared=prepared)
         if i >= args.warmup:
             per_step.append(gbs)
             reqs = n
