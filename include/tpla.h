@@ -185,9 +185,15 @@ TPLA_API int tpla_decode(const tpla_tensor* q, const tpla_tensor* kv_cache,
  * This call never calls cudaMalloc, cudaFree or any allocating routine.
  *   - A problem whose workspace (tpla_decode_workspace_size) exceeds that
  *     capacity is rejected with TPLA_ERR_WORKSPACE before any launch.
- *   - The first call on a device looks up the buffer's device address
- *     (cudaGetSymbolAddress, once per device, with that device current);
- *     make that first call before capturing a stream.
+ *   - The first valid call on a device is its set-up call: it looks up the
+ *     buffer's device address (cudaGetSymbolAddress, once per device, with
+ *     that device current).  Under CUDA's lazy module loading (the default)
+ *     that lookup is also what loads the buffer, so the first call may
+ *     reserve TPLA_NOALLOC_SCRATCH_BYTES of device memory.  Make one call
+ *     on each device before handing its memory to an arena or pool and
+ *     before capturing a stream; later calls reserve nothing.
+ *   - The address is kept for the life of the process: do not use the
+ *     library on a device after cudaDeviceReset on it.
  *   - All calls on a device share the one buffer and it keeps the previous
  *     call's contents (nothing needs clearing: every entry read is written
  *     earlier in the same call).  Calls whose kernels overlap on the GPU,
@@ -260,7 +266,6 @@ TPLA_API int tpla_get_device_status(tpla_stream_t stream, int* status);
  * inside a timed region. */
 TPLA_API int64_t tpla_launch_count(void);
 
-/* TPLA_VERSION of the loaded library. */
 /*
  * tpla_selftest_wait_timeout -- test support for the device failure path;
  * the pages have no counterpart.  Launches one thread that waits, through
@@ -272,6 +277,7 @@ TPLA_API int64_t tpla_launch_count(void);
  */
 TPLA_API int tpla_selftest_wait_timeout(int microseconds, tpla_stream_t stream);
 
+/* TPLA_VERSION of the loaded library. */
 TPLA_API int tpla_version(void);
 
 #ifdef __cplusplus

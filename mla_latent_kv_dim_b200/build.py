@@ -65,7 +65,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         list(ex.map(run, jobs))
     if force or jobs or _stale(LIB, objs):
         run([nvcc, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs,
-             "-Xlinker", "--no-undefined", "-lcuda" if False else "-ldl"])
+             "-Xlinker", "--no-undefined", "-ldl"])
     return LIB
 
 

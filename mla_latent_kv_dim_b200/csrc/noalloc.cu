@@ -7,7 +7,10 @@
 // slow.  For them this entry point takes no workspace argument and never
 // allocates: the split-KV partial results live in one file-scope __device__
 // array, reserved when the library's code is loaded on a device and kept
-// there until the process exits.
+// there until the process exits.  Under CUDA's lazy module loading that
+// load happens at the first call on a device (the symbol lookup below), so
+// the first call is the set-up call: it may reserve the buffer; later calls
+// reserve nothing.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -29,7 +32,9 @@ void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device.  In host code
 // the symbol itself is only a handle; cudaGetSymbolAddress turns it into a
-// pointer kernels may use.  Looked up once per device and cached.
+// pointer kernels may use.  Looked up once per device and cached; the cached
+// address belongs to the device's current context, so the library must not
+// be used across cudaDeviceReset (the buffer may be placed elsewhere after).
 int scratch_for_current_device(void** ptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -66,10 +71,13 @@ extern "C" int tpla_decode_noalloc(const tpla_tensor* q, const tpla_tensor* kv_c
                                       &opts, &need);
   if (rc != TPLA_OK) return rc;
   if (need > tpla::kScratchBytes) return TPLA_ERR_WORKSPACE;  // beyond the fixed capacity
+  // The set-up (symbol lookup, which also loads the buffer) runs on the first
+  // valid call on a device whether or not that call needs scratch, so that
+  // "make one call first" is enough for every later call.
+  void* ws = nullptr;
+  rc = tpla::scratch_for_current_device(&ws);
+  if (rc != TPLA_OK) return rc;
   if (need > 0) {
-    void* ws = nullptr;
-    rc = tpla::scratch_for_current_device(&ws);
-    if (rc != TPLA_OK) return rc;
     opts.workspace = ws;
     opts.workspace_bytes = tpla::kScratchBytes;
   }

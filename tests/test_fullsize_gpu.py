@@ -54,6 +54,29 @@ def test_dsv3_mla_g1_sampled(cuda_dev, dsv3):
     check_requests(w, out, lse, [0, 41], 1, "replicate")
 
 
+@pytest.mark.parametrize("G,rope,shard", [(2, "replicate", 0), (2, "replicate", 1),
+                                          (4, "replicate", 3), (4, "split", 1)])
+def test_dsv3_one_shard_sampled(cuda_dev, dsv3, G, rope, shard):
+    """One-shard mode (the bytes one tensor-parallel rank reads) on the whole
+    DeepSeek-V3-shaped workload, in the launch configuration the benchmark
+    times: every CTA pair walks several requests, so the query is reloaded
+    between segments.  Sampled requests, all heads and tokens, element by
+    element against the oracle's shard."""
+    w = dsv3
+    d = to_device(w, cuda_dev)
+    out_t, lse_t = tp.decode(d["q"], d["cache"], d["seq_lens"], d["page_table"], G, rope,
+                             w.scale, shard=shard)
+    torch.cuda.synchronize()
+    assert tp.device_status() == 0
+    out, lse = to_np(out_t), to_np(lse_t)
+    assert out.shape == (w.B, w.H, 512 // G) and lse.shape == (w.B, w.H, 1)
+    reqs = [0, 29, 63]
+    ro, rl = O.tpla_decode_ref(as_f64(w.q)[reqs], oracle_rows(w, reqs), G, rope,
+                               np.float32(w.scale), shard)
+    assert_out_close(out[reqs], ro)
+    assert_lse_close(lse[reqs], rl)
+
+
 def test_dsv3_tpla_g2_hadamard_step_sampled(cuda_dev, dsv3):
     """The benchmark step: Hadamard-rotated q and cache, TPLA G=2 decode, V-up
     with the rotation folded into W_uv.  The oracle rotates the same bf16

@@ -512,3 +512,26 @@ def test_pins_catch_planted_mistakes(monkeypatch):
         out, lse = O.mla_decode_ref(q, rows, SCALE)
         assert not np.allclose(out[0], np.array(ob), atol=1e-9)
     monkeypatch.setattr(O, "attention_ref", good)
+
+
+def test_per_head_cosine_hand_computed():
+    """The referee's fidelity measure (per-head cosine of two outputs), pinned
+    on rows whose cosines are known by hand: parallel (different lengths),
+    orthogonal, antiparallel, a 3-4-5 pair, a known angle, and a zero row
+    (defined as 0).  Each (request, head) is reduced over the last axis only."""
+    a = np.zeros((2, 3, 4))
+    b = np.zeros((2, 3, 4))
+    a[0, 0, :3], b[0, 0, :3] = [1, 2, 2], [2, 4, 4]          # parallel: 1
+    a[0, 1, :3], b[0, 1, :3] = [1, 0, 0], [0, 3, 0]          # orthogonal: 0
+    a[0, 2, :2], b[0, 2, :2] = [1, -1], [-2, 2]              # antiparallel: -1
+    a[1, 0, :2], b[1, 0, :2] = [3, 4], [8, 6]                # 48 / (5 * 10)
+    t = 0.3
+    a[1, 1, 2:], b[1, 1, 2:] = [math.cos(t), math.sin(t)], [5, 0]  # angle t
+    a[1, 2, :], b[1, 2, :] = [0, 0, 0, 0], [1, 1, 1, 1]      # zero row: 0
+    want = np.array([[1.0, 0.0, -1.0], [0.96, math.cos(t), 0.0]])
+    got = O.per_head_cosine(a, b)
+    assert got.shape == (2, 3)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-15)
+    # symmetric, and invariant under positive scaling of either argument
+    np.testing.assert_allclose(O.per_head_cosine(b, a), want, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(O.per_head_cosine(7.0 * a, 0.5 * b), want, rtol=0, atol=1e-15)

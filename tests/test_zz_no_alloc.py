@@ -1,8 +1,10 @@
 """tpla_decode_noalloc: the decode entry point for callers that cannot
 allocate device memory while they decode (its split-KV scratch is a fixed
 buffer the library reserves when it is loaded).  Checked through the C ABI
-against tpla_decode_ex, which takes caller-allocated workspace, on two calls
-in a row that both need scratch.  Kept in a file of its own, collected last."""
+against tpla_decode_ex, which takes caller-allocated workspace, and against
+the float64 oracle, on two calls in a row that both need scratch; a call
+after the first must not change the device's free memory.  Kept in a file of
+its own, collected last."""
 
 import ctypes
 
@@ -12,7 +14,8 @@ import torch
 import mla_latent_kv_dim_b200 as tp
 from mla_latent_kv_dim_b200 import _native as N
 from mla_latent_kv_dim_b200.workloads import make_inputs
-from parity import assert_lse_close, assert_out_close, to_device, to_np
+from parity import (assert_lse_close, assert_out_close, oracle_decode, to_device,
+                    to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -50,6 +53,7 @@ def test_noalloc_matches_decode_ex_twice(cuda_dev, case):
     assert 0 < need <= SCRATCH_LIMIT  # the case really uses scratch
     ref_out, ref_lse = tp.decode(d["q"], d["cache"], d["seq_lens"], d["page_table"], G, rope,
                                  w.scale, num_splits=case["splits"], shard=shard)
+    ora_out, ora_lse = oracle_decode(w, G, rope, shard=shard)
     for call in range(2):
         out = torch.full((w.B, w.H, width), float("nan"), device=cuda_dev)
         lse = torch.full((w.B, w.H, nsh), float("nan"), device=cuda_dev)
@@ -58,6 +62,24 @@ def test_noalloc_matches_decode_ex_twice(cuda_dev, case):
         torch.cuda.synchronize()
         assert_out_close(to_np(out), to_np(ref_out), what=f"call {call}")
         assert_lse_close(to_np(lse), to_np(ref_lse), what=f"call {call}")
+        assert_out_close(to_np(out), ora_out, what=f"call {call} vs oracle")
+        assert_lse_close(to_np(lse), ora_lse, what=f"call {call} vs oracle")
+
+
+def test_noalloc_reserves_nothing_after_its_first_call(cuda_dev):
+    """The first call on a device is the set-up call (it may load the fixed
+    buffer); a later call must leave the device's free memory unchanged."""
+    w = make_inputs(3, 64, [900, 64, 333], paged=True, decay=True, seed=7)
+    d = to_device(w, cuda_dev)
+    out = torch.empty((w.B, w.H, 512), device=cuda_dev)
+    lse = torch.empty((w.B, w.H, 2), device=cuda_dev)
+    assert _noalloc(d, 2, "replicate", w.scale, out, lse, 3) == 0
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    assert _noalloc(d, 2, "replicate", w.scale, out, lse, 3) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_dev):
