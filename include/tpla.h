@@ -71,8 +71,9 @@ enum tpla_status {
 enum tpla_rope_mode { TPLA_ROPE_REPLICATE = 0, TPLA_ROPE_SPLIT = 1 };
 
 enum tpla_kernel_choice {
-  TPLA_KERNEL_AUTO = 0,     /* tensor-core kernel where the shape allows it   */
-  TPLA_KERNEL_GENERIC = 1,  /* portable CUDA-core kernel (any supported shape) */
+  TPLA_KERNEL_AUTO = 0,     /* the tcgen05/TMA kernel (same as SM100)          */
+  TPLA_KERNEL_GENERIC = 1,  /* portable CUDA-core kernel, only when named: a   */
+                            /* reference point and the path for G = 8          */
   TPLA_KERNEL_SM100 = 2     /* tcgen05/TMA kernel; UNSUPPORTED if it cannot   */
 };
 
@@ -131,9 +132,13 @@ typedef struct {
  * values.  The tensor-core path reads whole pages and gives those rows zero
  * weight after the softmax, and 0 * NaN is NaN.
  *
- * Kernel choice (opts->kernel = AUTO): the tcgen05 kernel when the device is
- * sm_100, G is 1, 2 or 4, H <= 128, scale > 0 and out rows are 16-byte
- * aligned; the portable kernel otherwise.  Both compute the same function.
+ * Kernel choice (opts->kernel = AUTO or SM100): the tcgen05 kernel, which
+ * needs an sm_100 device, G of 1, 2 or 4 and out rows on 16-byte boundaries
+ * (data 16-byte aligned, stride[0] and stride[1] multiples of 16 bytes);
+ * otherwise TPLA_ERR_UNSUPPORTED before any launch.  Any finite scale
+ * (negative and zero included) and any H (one launch per group of 128
+ * heads) are taken.  The portable kernel (opts->kernel = GENERIC) computes
+ * the same function and runs only when named.
  *
  * Size limits (TPLA_ERR_UNSUPPORTED beyond them, nothing launched):
  * B <= 2^20, H <= 4096, B * H <= 2^30, num_splits <= 65535,
@@ -148,10 +153,7 @@ TPLA_API int tpla_decode_ex(const tpla_tensor* q, const tpla_tensor* kv_cache,
 /*
  * tpla_decode_workspace_size -- bytes of device workspace tpla_decode_ex
  * needs for these arguments and options (0 when no split is used).  Same
- * validation as tpla_decode_ex; writes the size to *bytes.  With
- * TPLA_KERNEL_AUTO the size covers either kernel, because the automatic
- * choice also depends on the scale, which this query does not take (a
- * scale <= 0 runs the generic kernel).
+ * validation as tpla_decode_ex; writes the size to *bytes.
  */
 TPLA_API int tpla_decode_workspace_size(const tpla_tensor* q, const tpla_tensor* kv_cache,
                                const tpla_tensor* seq_lens,

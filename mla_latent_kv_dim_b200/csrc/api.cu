@@ -149,7 +149,10 @@ int choose_path(const DecodeProblem& p, const tpla_decode_opts* opts, Path* path
     if (!fast) return TPLA_ERR_UNSUPPORTED;
     *path = Path::Sm100;
   } else {
-    *path = fast ? Path::Sm100 : Path::Generic;
+    // the automatic choice is the tcgen05 kernel; the portable kernel runs
+    // only when the caller names it
+    if (!fast) return TPLA_ERR_UNSUPPORTED;
+    *path = Path::Sm100;
   }
   if (*path == Path::Generic && (int64_t)p.B * p.n_shards > kMaxGenericRequestShards)
     return TPLA_ERR_UNSUPPORTED;
@@ -213,18 +216,7 @@ int tpla_decode_workspace_size(const tpla_tensor* q, const tpla_tensor* kv_cache
   Path path;
   rc = choose_path(p, opts, &path);
   if (rc != TPLA_OK) return rc;
-  rc = workspace_needed(p, opts, path, bytes);
-  if (rc != TPLA_OK) return rc;
-  // The automatic choice also depends on the scale, which this query does not
-  // take (a scale <= 0 runs the generic kernel), so size for either kernel.
-  const int choice = opts ? opts->kernel : TPLA_KERNEL_AUTO;
-  if (choice == TPLA_KERNEL_AUTO && path == Path::Sm100) {
-    size_t g = 0;
-    rc = workspace_needed(p, opts, Path::Generic, &g);
-    if (rc != TPLA_OK) return rc;
-    if (g > *bytes) *bytes = g;
-  }
-  return TPLA_OK;
+  return workspace_needed(p, opts, path, bytes);
 }
 
 int tpla_decode_ex(const tpla_tensor* q, const tpla_tensor* kv_cache,
@@ -329,7 +321,10 @@ int tpla_vup_combine(const tpla_tensor* out_latent, const tpla_tensor* W_uv, tpl
   if (Dv % 16 != 0 || Dv < 16 || Dv > 256) return TPLA_ERR_UNSUPPORTED;
   if (!check_tensor(y, TPLA_F32, 3) || y->shape[0] != B || y->shape[1] != H || y->shape[2] != Dv)
     return TPLA_ERR_INVALID_ARG;
-  if (H > 65535) return TPLA_ERR_UNSUPPORTED;
+  if (H > 65535 || (B + 63) / 64 > 65535) return TPLA_ERR_UNSUPPORTED;
+  if (!vup_supported(out_latent->data, out_latent->dtype == TPLA_BF16, out_latent->stride[0],
+                     out_latent->stride[1], W_uv->data, W_uv->stride[0], W_uv->stride[1]))
+    return TPLA_ERR_UNSUPPORTED;
   cudaError_t e = launch_vup(out_latent->data, out_latent->dtype == TPLA_BF16,
                              out_latent->stride[0], out_latent->stride[1], W_uv->data,
                              W_uv->stride[0], W_uv->stride[1],
@@ -362,7 +357,10 @@ int tpla_get_device_status(tpla_stream_t stream, int* status) {
   if (e != cudaSuccess) return cuda_fail(e);
   e = status_read_clear_sm100(&b);
   if (e != cudaSuccess) return cuda_fail(e);
-  *status = a != 0 ? a : b;
+  int c = 0;
+  e = status_read_clear_vup(&c);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *status = a != 0 ? a : (b != 0 ? b : c);
   return TPLA_OK;
 }
 

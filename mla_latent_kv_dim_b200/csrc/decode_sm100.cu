@@ -123,7 +123,8 @@ struct Params {
   int NB;    // PV block width: min(256, d) latent columns per MMA
   int nblk;  // PV blocks per shard (d / NB)
   int qk_slots, pv_slots;  // ring split (sum kRingSlots)
-  float scale_log2;  // softmax scale * log2(e)
+  float scale_log2;  // |softmax scale| * log2(e) (> 0; see the launcher)
+  int negate;        // scale < 0: the scores are negated before the softmax
   void* out;
   int out_bf16;
   int64_t o_sb, o_sh;
@@ -745,13 +746,18 @@ __device__ void softmax_warps(const Params& p, int cl, uint32_t rank, uint32_t s
       tc_fence_before();
       __syncwarp();
       if ((tid & 31) == 0) mbar_arrive_remote(sf_c[Ug & 1]);
-      // raw scores; the positive scale is applied inside the exponent
+      // raw scores; |scale| is applied inside the exponent, a negative
+      // scale's sign here (uniform branch, not taken for the usual scale > 0)
       const int nv = max(0, min(64, s.L - (kTileTok * t + 128 * half + 64 * wg)));
       float x[64];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         x[j] = __uint_as_float(r0[j]);
         x[j + 32] = __uint_as_float(r1[j]);
+      }
+      if (p.negate) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) x[j] = -x[j];
       }
       if (nv < 64) {  // warp-uniform: a warp covers one 64-token range
 #pragma unroll
@@ -918,60 +924,96 @@ tpla_decode_sm100_kernel(const __grid_constant__ CUtensorMap qmap,
 }
 
 // ---------------------------------------------------------------- merge of partial slots
+//
+// Requests cut by a range boundary (or explicitly split) left normalised
+// partial outputs and their lse in workspace slots; the exact log-sum-exp
+// rule combines them.  A block covers one request and kMergeHeads heads, one
+// warp per head: the lanes hold the slots' lse (32 at a time) and 16-byte
+// column groups, so every warp keeps several independent loads in flight.
+// Requests that one cluster finished (written final by the decode kernel)
+// return after the block's prefix sum.
 
-constexpr int kMergeThreads = 128;
+constexpr int kMergeHeads = 8;
+constexpr int kMergeThreads = 32 * kMergeHeads;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
 
 __global__ void __launch_bounds__(kMergeThreads)
 sm100_merge_kernel(const Params p) {
-  const int b = blockIdx.x / p.H;
-  const int h = blockIdx.x % p.H;
-  __shared__ long long red[2][kMergeThreads];
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * kMergeHeads + warp;
+  __shared__ long long red[2][kMergeHeads];
   long long pre = 0, tot = 0;
-  for (int bb = threadIdx.x; bb < p.B; bb += kMergeThreads) {
-    const long long nt = req_tiles(p, bb);
-    tot += nt;
-    if (bb < b) pre += nt;
-  }
-  red[0][threadIdx.x] = pre;
-  red[1][threadIdx.x] = tot;
-  __syncthreads();
-  for (int o = kMergeThreads / 2; o; o >>= 1) {
-    if (threadIdx.x < o) {
-      red[0][threadIdx.x] += red[0][threadIdx.x + o];
-      red[1][threadIdx.x] += red[1][threadIdx.x + o];
+  if (p.mode == 0) {  // tiles before request b and in total
+    for (int bb = threadIdx.x; bb < p.B; bb += kMergeThreads) {
+      const long long nt = req_tiles(p, bb);
+      tot += nt;
+      if (bb < b) pre += nt;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      pre += __shfl_xor_sync(0xffffffffu, pre, o);
+      tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    }
+    if (lane == 0) {
+      red[0][warp] = pre;
+      red[1][warp] = tot;
     }
     __syncthreads();
+    pre = tot = 0;
+    for (int w = 0; w < kMergeHeads; ++w) {
+      pre += red[0][w];
+      tot += red[1][w];
+    }
   }
-  pre = red[0][0];
-  const long long T = red[1][0];
+  const long long T = tot;
   const int nt = req_tiles(p, b);
-  const int cw = p.W / p.nsh;
-
-  auto write_final = [&](int k, int col, float v) {
-    const int64_t off = (int64_t)b * p.o_sb + (int64_t)h * p.o_sh + k * cw + col;
-    if (p.out_bf16)
-      reinterpret_cast<__nv_bfloat16*>(p.out)[off] = __float2bfloat16_rn(v);
-    else
-      reinterpret_cast<float*>(p.out)[off] = v;
+  int s_lo = 0, s_hi = 0;  // cluster range of request b
+  const long long P = min((long long)p.P, T);  // clusters that received work
+  if (nt > 0) {
+    if (p.mode == 0) {
+      s_lo = (int)(((pre + 1) * P + T - 1) / T - 1);
+      s_hi = (int)(((pre + nt) * P + T - 1) / T - 1);
+      if (s_lo == s_hi) return;  // one cluster wrote the final result
+    } else {
+      if (p.S == 1) return;
+      s_lo = b * p.S;
+      s_hi = b * p.S + p.S - 1;
+    }
+  }
+  if (h >= p.H) return;
+  const int cw = p.W / p.nsh;  // columns per shard (a multiple of 64)
+  auto write4 = [&](int col, float4 v) {
+    const int64_t off = (int64_t)b * p.o_sb + (int64_t)h * p.o_sh + col;
+    if (p.out_bf16) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t*>(&lo);
+      w.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + off) = w;
+    } else {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + off) = v;
+    }
   };
-
-  if (nt == 0) {  // empty request
+  auto write_lse = [&](int k, float v) {
+    if (p.lse && lane == 0) p.lse[(int64_t)b * p.l_sb + (int64_t)h * p.l_sh + k] = v;
+  };
+  if (nt == 0) {  // empty request: never reached by the decode kernel
     for (int k = 0; k < p.nsh; ++k) {
-      for (int c = threadIdx.x; c < cw; c += kMergeThreads) write_final(k, c, 0.f);
-      if (p.lse && threadIdx.x == 0) p.lse[(int64_t)b * p.l_sb + (int64_t)h * p.l_sh + k] = -INFINITY;
+      for (int c = 4 * lane; c < cw; c += 128) write4(k * cw + c, make_float4(0.f, 0.f, 0.f, 0.f));
+      write_lse(k, -INFINITY);
     }
     return;
-  }
-  int s_lo, s_hi;  // cluster range
-  const long long P = min((long long)p.P, T);  // clusters that received work
-  if (p.mode == 0) {
-    s_lo = (int)(((pre + 1) * P + T - 1) / T - 1);
-    s_hi = (int)(((pre + nt) * P + T - 1) / T - 1);
-    if (s_lo == s_hi) return;  // one cluster wrote the final result
-  } else {
-    if (p.S == 1) return;
-    s_lo = b * p.S;
-    s_hi = b * p.S + p.S - 1;
   }
   auto slot_of = [&](int c) -> int {
     if (p.mode == 0) {
@@ -980,29 +1022,69 @@ sm100_merge_kernel(const Params p) {
     }
     return 2 * c;
   };
+  // Column groups of this lane: 16-byte groups 4 * lane + 128 * i of each
+  // shard (cw <= 512, so at most four).  Loads of two slots x all groups go
+  // out together before the multiply-adds.
+  const int ngrp = (cw + 127) / 128;
   for (int k = 0; k < p.nsh; ++k) {
+    auto lse_of = [&](int c) { return __ldcg(p.part_l + ((int64_t)slot_of(c) * p.H + h) * p.nsh + k); };
+    auto row_of = [&](int c) {
+      return reinterpret_cast<const float4*>(p.part_o + ((int64_t)slot_of(c) * p.H + h) * p.W +
+                                             k * cw) + lane;
+    };
     float M = -INFINITY;
-    for (int c = s_lo; c <= s_hi; ++c)
-      M = fmaxf(M, p.part_l[((int64_t)slot_of(c) * p.H + h) * p.nsh + k]);
+    for (int c = s_lo + lane; c <= s_hi; c += 32) M = fmaxf(M, lse_of(c));
+    M = warp_max(M);
     float z = 0.f;
     if (M != -INFINITY)
-      for (int c = s_lo; c <= s_hi; ++c) {
-        const float ls = p.part_l[((int64_t)slot_of(c) * p.H + h) * p.nsh + k];
-        if (ls != -INFINITY) z += expf(ls - M);
+      for (int c = s_lo + lane; c <= s_hi; c += 32) {
+        const float ls = lse_of(c);
+        z += ls == -INFINITY ? 0.f : expf(ls - M);
       }
+    z = warp_sum(z);
     const float total = M == -INFINITY ? -INFINITY : M + logf(z);
-    for (int col = threadIdx.x; col < cw; col += kMergeThreads) {
-      float acc = 0.f;
-      if (total != -INFINITY)
-        for (int c = s_lo; c <= s_hi; ++c) {
-          const int sl = slot_of(c);
-          const float ls = p.part_l[((int64_t)sl * p.H + h) * p.nsh + k];
-          if (ls == -INFINITY) continue;
-          acc = fmaf(expf(ls - total), p.part_o[((int64_t)sl * p.H + h) * p.W + k * cw + col], acc);
+    float4 acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (total != -INFINITY) {
+      for (int g0 = s_lo; g0 <= s_hi; g0 += 32) {
+        float wmine = 0.f;
+        if (g0 + lane <= s_hi) {
+          const float ls = lse_of(g0 + lane);
+          wmine = ls == -INFINITY ? 0.f : expf(ls - total);
         }
-      write_final(k, col, acc);
+        const int n = min(32, s_hi - g0 + 1);
+        for (int i0 = 0; i0 < n; i0 += 2) {
+          const float w0 = __shfl_sync(0xffffffffu, wmine, i0);
+          const float w1 = __shfl_sync(0xffffffffu, wmine, min(i0 + 1, 31));
+          const bool has1 = i0 + 1 < n && w1 != 0.f;
+          const float4* r0 = row_of(g0 + i0);
+          const float4* r1 = has1 ? row_of(g0 + i0 + 1) : r0;
+          float4 o0[4], o1[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (i < ngrp && 4 * lane + 128 * i < cw) {
+              o0[i] = w0 != 0.f ? __ldcg(r0 + 32 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+              o1[i] = has1 ? __ldcg(r1 + 32 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          }
+          const float v1 = has1 ? w1 : 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (i < ngrp && 4 * lane + 128 * i < cw) {
+              acc[i].x = fmaf(v1, o1[i].x, fmaf(w0, o0[i].x, acc[i].x));
+              acc[i].y = fmaf(v1, o1[i].y, fmaf(w0, o0[i].y, acc[i].y));
+              acc[i].z = fmaf(v1, o1[i].z, fmaf(w0, o0[i].z, acc[i].z));
+              acc[i].w = fmaf(v1, o1[i].w, fmaf(w0, o0[i].w, acc[i].w));
+            }
+          }
+        }
+      }
     }
-    if (p.lse && threadIdx.x == 0) p.lse[(int64_t)b * p.l_sb + (int64_t)h * p.l_sh + k] = total;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i < ngrp && 4 * lane + 128 * i < cw) write4(k * cw + 4 * lane + 128 * i, acc[i]);
+    write_lse(k, total);
   }
 }
 
@@ -1034,6 +1116,22 @@ std::mutex g_mu;
 DeviceInfo g_dev[64];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// cuTensorMapEncodeTiled from the driver (looked up once; g_mu held).
+void* encoder_locked() {
+  static void* fn = nullptr;
+  if (fn) return fn;
+  void* f = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !f) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  fn = f;
+  return fn;
+}
+
 cudaError_t launch_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int clusters,
                           cudaStream_t stream) {
   cfg = {};
@@ -1063,15 +1161,8 @@ const DeviceInfo& device_info(int dev) {
   }
   if (major != 10 || minor != 0) return d;
   if (!g_encode) {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !fn) {
-      cudaGetLastError();
-      return d;
-    }
-    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(encoder_locked());
+    if (!g_encode) return d;
   }
   if (cudaFuncSetAttribute(tpla_decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSmemBytes) != cudaSuccess) {
@@ -1130,12 +1221,21 @@ int num_slots(const DecodeProblem& p, int num_splits, int max_clusters) {
 
 }  // namespace
 
+void* tensor_map_encoder() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  return encoder_locked();
+}
+
+bool sm100_device(int device) {
+  if (device < 0 || device >= 64) return false;
+  return device_info(device).sm100;
+}
+
 bool sm100_supported(const DecodeProblem& p, int device) {
   if (device < 0 || device >= 64) return false;
   if (!(p.G == 1 || p.G == 2 || p.G == 4)) return false;
-  if (p.H < 1 || p.H > 128) return false;
-  // the kernel takes the row max of raw scores and scales inside exp2
-  if (!(p.scale > 0.f) || !isfinite(p.scale)) return false;
+  if (p.H < 1) return false;  // more than 128 heads: one launch per 128-head group
+  if (!isfinite(p.scale)) return false;
   if (p.cache_rows > (1 << 30) || (p.page_table && p.num_blocks >= (1LL << 31) - 1)) return false;
   if (p.page_table && p.max_pages > (1 << 24)) return false;
   // 16-byte vector stores of out rows
@@ -1149,12 +1249,32 @@ size_t sm100_workspace_bytes(const DecodeProblem& p, int num_splits, int device)
   const DeviceInfo& d = device_info(device);
   const int slots = num_slots(p, num_splits, d.max_clusters);
   if (slots == 0) return 0;
-  const size_t o = (size_t)slots * p.H * p.out_width * sizeof(float);
-  return ((o + 255) / 256) * 256 + (size_t)slots * p.H * p.n_shards * sizeof(float);
+  const size_t Hg = p.H < 128 ? p.H : 128;  // heads of one launch (128-head groups)
+  const size_t o = (size_t)slots * Hg * p.out_width * sizeof(float);
+  return ((o + 255) / 256) * 256 + (size_t)slots * Hg * p.n_shards * sizeof(float);
 }
 
+cudaError_t launch_decode_sm100_group(const DecodeProblem& dp, int num_splits, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream);
+
+// More than 128 heads: one launch (plus merge) per group of up to 128 heads,
+// in stream order, reusing the same workspace.
 cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* ws, size_t ws_bytes,
                                 cudaStream_t stream) {
+  for (int h0 = 0; h0 < dp.H; h0 += 128) {
+    DecodeProblem g = dp;
+    g.H = dp.H - h0 < 128 ? dp.H - h0 : 128;
+    g.q = reinterpret_cast<const __nv_bfloat16*>(dp.q) + (int64_t)h0 * dp.q_sh;
+    g.out = reinterpret_cast<char*>(dp.out) + (int64_t)h0 * dp.o_sh * (dp.out_bf16 ? 2 : 4);
+    g.lse = dp.lse ? dp.lse + (int64_t)h0 * dp.l_sh : nullptr;
+    cudaError_t e = launch_decode_sm100_group(g, num_splits, ws, ws_bytes, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode_sm100_group(const DecodeProblem& dp, int num_splits, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream) {
   int dev = 0;
   cudaGetDevice(&dev);
   const DeviceInfo& d = device_info(dev);
@@ -1192,7 +1312,12 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
   // measured: G=1 (eight PV stages per tile) wants the deeper PV ring
   p.qk_slots = dp.G == 1 ? 3 : 4;
   p.pv_slots = kRingSlots - p.qk_slots;
-  p.scale_log2 = (float)((double)dp.scale * 1.4426950408889634);
+  // The kernel takes the row max of the sign-corrected raw scores and applies
+  // |scale| inside exp2.  A zero scale becomes 1e-30 (log2 units): every
+  // finite score then gives exp2(~0) = 1 exactly in f32, as scale 0 does,
+  // while masked (-inf) scores still give 0.
+  p.scale_log2 = fmaxf((float)(fabs((double)dp.scale) * 1.4426950408889634), 1e-30f);
+  p.negate = dp.scale < 0.f;
   p.out = dp.out;
   p.out_bf16 = dp.out_bf16;
   p.o_sb = dp.o_sb;
@@ -1228,7 +1353,8 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
   count_launch();
   if (e != cudaSuccess) return e;
   if (p.mode == 0 || p.S > 1) {
-    sm100_merge_kernel<<<dp.B * dp.H, kMergeThreads, 0, stream>>>(p);
+    sm100_merge_kernel<<<dim3(dp.B, (dp.H + kMergeHeads - 1) / kMergeHeads), kMergeThreads, 0,
+                         stream>>>(p);
     count_launch();
     e = cudaGetLastError();
   }

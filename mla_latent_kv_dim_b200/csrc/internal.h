@@ -50,6 +50,10 @@ cudaError_t launch_decode_generic(const DecodeProblem& p, int splits, void* ws,
                                   cudaStream_t stream);
 
 // ---------------------------------------------------------------- sm100 path
+// cuTensorMapEncodeTiled (as void*), or nullptr when the driver lacks it.
+void* tensor_map_encoder();
+// True when `device` is an sm_100 GPU the tcgen05 kernels can run on.
+bool sm100_device(int device);
 // Returns true when the tcgen05 kernel can run this problem on this device.
 bool sm100_supported(const DecodeProblem& p, int device);
 size_t sm100_workspace_bytes(const DecodeProblem& p, int num_splits, int device);
@@ -69,6 +73,10 @@ cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int S
 // ---------------------------------------------------------------- hadamard / vup
 cudaError_t launch_hadamard(void* buf, int bf16, int ndim, const int64_t* shape,
                             const int64_t* stride, int dim, cudaStream_t stream);
+// True when the V-up kernel takes these layouts (TMA: 16-byte aligned bases
+// and row strides).
+bool vup_supported(const void* out_latent, int out_bf16, int64_t o_sb, int64_t o_sh,
+                   const void* W, int64_t w_sh, int64_t w_sj);
 cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64_t o_sh,
                        const void* W, int64_t w_sh, int64_t w_sj, float* y,
                        int64_t y_sb, int64_t y_sh, int B, int H, int Dv,
@@ -83,6 +91,7 @@ void count_launch(int n = 1);
 // these read and clear it (after the caller synchronised the stream).
 cudaError_t status_read_clear_generic(int* code);
 cudaError_t status_read_clear_sm100(int* code);
+cudaError_t status_read_clear_vup(int* code);
 cudaError_t launch_wait_timeout_selftest(long long cycles, cudaStream_t stream);
 
 }  // namespace tpla

@@ -6,320 +6,408 @@
 // side by side in latent space, the sum over shards is exactly the
 // contraction over j here, so this kernel stands in for that all-reduce.
 //
-// Per head h this is a small GEMM [B x 512] x [512 x Dv].  It is bound by
-// reading W_uv (H * 512 * Dv bf16) and out (B * H * 512 f32) once.  Tensor
-// cores (bf16 in, f32 accumulate); an f32 `out` is split into hi + lo bf16
-// terms, so the result keeps about 16 mantissa bits of `out`.
-//
-// The tiled kernel (16-byte aligned operands) gives every CTA a 64 x 64
-// output tile of one head, streams K in chunks of 64 with the next chunk's
-// global loads in flight while the current one is multiplied, and reads
-// fragments with ldmatrix from padded (conflict-free) shared-memory rows.
-// Other layouts take the element-wise kernel.
+// Per head h this is a small GEMM, computed transposed on the 5th-generation
+// tensor core:  Y_h^T [Dv x B] = W_h^T [Dv x 512] . out_h^T [512 x B], so the
+// MMA's M is the V dimension (128 per accumulator, two accumulators for
+// Dv > 128) and N the batch tile (up to 64 requests).  The op reads W_uv
+// (H * 512 * Dv bf16) and out (B * H * 512, f32 or bf16) once and is bound by
+// HBM; what matters is many bytes in flight per SM:
+//  * one CTA per (head, batch tile); W and out arrive by TMA (no multicast)
+//    in 64-column K chunks through a ring of up to 8 stages (~160 KB in
+//    flight per SM);
+//  * W lands MN-major in the 128-byte swizzle the MMA reads directly; a bf16
+//    `out` lands K-major the same way; an f32 `out` lands as plain rows and
+//    four converter warps split it into hi + lo bf16 tiles (out = hi + lo to
+//    about 16 mantissa bits), each multiplied by the same W tile;
+//  * one thread issues the tcgen05 MMAs into TMEM; the converter warps read
+//    the accumulators back and store y.
+// Every barrier wait is bounded; on timeout the kernel records
+// TPLA_ERR_DEVICE_TIMEOUT in its status word and stops.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace tpla {
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kMTile = 16 * kWarps;  // rows of B per CTA
-constexpr int kKChunk = 32;
-constexpr int kRowWords = kKChunk / 2 + 4;  // padded smem row, 32-bit words
+using namespace ptx;
 
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4],
-                                               uint32_t b0, uint32_t b1) {
+constexpr int kKC = 64;                   // latent columns per K chunk
+constexpr int kKChunks = kLatent / kKC;   // 8
+constexpr int kMaxN = 64;                 // batch rows per CTA (MMA N)
+constexpr int kWBox = 8192;               // one [64 j][64 v] bf16 tile
+constexpr int kConvStages = 2;
+constexpr int kMaxRaw = 8;
+constexpr int kThreads = 192;             // warp 0 TMA, warp 1 MMA, warps 2-5 convert + store
+constexpr int kSmemBudget = 200 * 1024;
+constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s at full clock
+
+__device__ int g_vup_status;
+
+struct VupParams {
+  float* y;
+  int64_t y_sb, y_sh;
+  int B, H, Dv;
+  int mh;          // 128-row halves of Dv (1 or 2)
+  int nt;          // batch rows per tile (MMA N), multiple of 16, <= 64
+  int out_bf16;
+  int raw_stages;
+  uint32_t raw_bytes;  // per stage: mh * 2 W tiles, then the out tile (1 KB aligned)
+  uint32_t tx_bytes;   // bytes the TMA copies of one stage deliver
+  uint32_t o_bytes;    // out tile bytes (nt rows of 64 values)
+  uint32_t off_conv, off_bar;
+};
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, uint32_t bar) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];"
+      :
+      : "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
-  return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      :
+      : "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
-template <int NT, bool OUT_BF16>  // NT = Dv / 8 n-tiles per warp
-__global__ void __launch_bounds__(kWarps * 32)
-vup_kernel(const void* __restrict__ outp, int64_t o_sb, int64_t o_sh,
-           const __nv_bfloat16* __restrict__ W, int64_t w_sh, int64_t w_sj,
-           float* __restrict__ y, int64_t y_sb, int64_t y_sh, int B) {
-  constexpr int Dv = NT * 8;
-  __shared__ uint32_t a_hi[kMTile][kRowWords];
-  __shared__ uint32_t a_lo[kMTile][kRowWords];
-  __shared__ uint32_t w_t[Dv][kRowWords];  // W chunk transposed: [n][k]
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
 
-  const int h = blockIdx.y;
-  const int m0 = blockIdx.x * kMTile;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gid = lane >> 2, t4 = lane & 3;
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 
-  float acc[NT][4];
-#pragma unroll
-  for (int n = 0; n < NT; ++n)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
-
-  for (int k0 = 0; k0 < kLatent; k0 += kKChunk) {
-    __syncthreads();
-    // A chunk: kMTile rows x 32 k, split into hi/lo bf16 pairs
-    for (int i = tid; i < kMTile * (kKChunk / 2); i += kWarps * 32) {
-      int r = i / (kKChunk / 2), kp = i % (kKChunk / 2);
-      int b = m0 + r;
-      float x0 = 0.f, x1 = 0.f;
-      if (b < B) {
-        int64_t off = (int64_t)b * o_sb + (int64_t)h * o_sh + k0 + 2 * kp;
-        if (OUT_BF16) {
-          const __nv_bfloat16* o = reinterpret_cast<const __nv_bfloat16*>(outp) + off;
-          x0 = __bfloat162float(o[0]);
-          x1 = __bfloat162float(o[1]);
-        } else {
-          const float* o = reinterpret_cast<const float*>(outp) + off;
-          x0 = o[0];
-          x1 = o[1];
-        }
-      }
-      __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-      a_hi[r][kp] = pack_bf16(h0, h1);
-      if (!OUT_BF16)
-        a_lo[r][kp] = pack_bf16(__float2bfloat16_rn(x0 - __bfloat162float(h0)),
-                                __float2bfloat16_rn(x1 - __bfloat162float(h1)));
-    }
-    // W chunk: 32 k rows x Dv, stored transposed as [n][k] pairs
-    for (int i = tid; i < (kKChunk / 2) * Dv; i += kWarps * 32) {
-      int kp = i / Dv, n = i % Dv;
-      const __nv_bfloat16* wp = W + (int64_t)h * w_sh + (int64_t)(k0 + 2 * kp) * w_sj + n;
-      w_t[n][kp] = pack_bf16(wp[0], wp[w_sj]);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kKChunk / 2; kk += 8) {  // two k16 steps (8 words each)
-      const int ra = warp * 16 + gid;
-      uint32_t ah[4] = {a_hi[ra][kk + t4], a_hi[ra + 8][kk + t4],
-                        a_hi[ra][kk + 4 + t4], a_hi[ra + 8][kk + 4 + t4]};
-      uint32_t al[4];
-      if (!OUT_BF16) {
-        al[0] = a_lo[ra][kk + t4];
-        al[1] = a_lo[ra + 8][kk + t4];
-        al[2] = a_lo[ra][kk + 4 + t4];
-        al[3] = a_lo[ra + 8][kk + 4 + t4];
-      }
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        uint32_t b0 = w_t[n * 8 + gid][kk + t4];
-        uint32_t b1 = w_t[n * 8 + gid][kk + 4 + t4];
-        mma_bf16_16816(acc[n], ah, b0, b1);
-        if (!OUT_BF16) mma_bf16_16816(acc[n], al, b0, b1);
+// Bounded wait; false on timeout (status recorded) or when another role
+// already gave up.
+__device__ bool wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
+    if ((i & 15) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kTimeoutCycles) {
+        atomicCAS(&g_vup_status, 0, TPLA_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+        return false;
       }
     }
   }
-  const int r0 = m0 + warp * 16 + gid;
-#pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    int c = n * 8 + 2 * t4;
-    if (r0 < B) {
-      float* yp = y + (int64_t)r0 * y_sb + (int64_t)h * y_sh + c;
-      yp[0] = acc[n][0];
-      yp[1] = acc[n][1];
+}
+
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+vup_sm100_kernel(const __grid_constant__ CUtensorMap wmap,
+                 const __grid_constant__ CUtensorMap omap, const VupParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x;
+  const int b0 = blockIdx.y * p.nt;
+  const int R = p.raw_stages;
+  const uint32_t bar0 = sbase + p.off_bar;
+  auto raw_full = [&](int s) { return bar0 + 8 * s; };
+  auto raw_empty = [&](int s) { return bar0 + 8 * (kMaxRaw + s); };
+  auto conv_full = [&](int c) { return bar0 + 8 * (2 * kMaxRaw + c); };
+  auto conv_empty = [&](int c) { return bar0 + 8 * (2 * kMaxRaw + kConvStages + c); };
+  const uint32_t acc_full = bar0 + 8 * (2 * kMaxRaw + 2 * kConvStages);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + p.off_bar + 8 * (2 * kMaxRaw + 2 * kConvStages + 1));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < R; ++s) {
+      mbar_init(raw_full(s), 1);
+      mbar_init(raw_empty(s), 1);
     }
-    if (r0 + 8 < B) {
-      float* yp = y + (int64_t)(r0 + 8) * y_sb + (int64_t)h * y_sh + c;
-      yp[0] = acc[n][2];
-      yp[1] = acc[n][3];
+    for (int c = 0; c < kConvStages; ++c) {
+      mbar_init(conv_full(c), 4);  // one arrival per converter warp
+      mbar_init(conv_empty(c), 1);
     }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-}
+  if (warp == 1) {  // accumulators: mh blocks of 64 columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(p.mh == 2 ? 128u : 64u)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-// ---------------------------------------------------------------- tiled kernel
-
-constexpr int kTM = 64, kTN = 64, kTK = 64;  // CTA tile: rows of B, columns of Dv, K chunk
-constexpr int kTRow = kTK + 8;               // padded smem row (bf16): 144 bytes
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                          uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-template <bool OUT_BF16>
-__global__ void __launch_bounds__(128)
-vup_tiled_kernel(const void* __restrict__ outp, int64_t o_sb, int64_t o_sh,
-                 const __nv_bfloat16* __restrict__ W, int64_t w_sh, int64_t w_sj,
-                 float* __restrict__ y, int64_t y_sb, int64_t y_sh, int B, int Dv) {
-  __shared__ __align__(16) __nv_bfloat16 a_hi[kTM][kTRow];
-  __shared__ __align__(16) __nv_bfloat16 a_lo[OUT_BF16 ? 1 : kTM][kTRow];
-  __shared__ __align__(16) __nv_bfloat16 w_s[kTK][kTRow];  // [k][n]
-
-  const int m0 = blockIdx.x * kTM, h = blockIdx.y, n0 = blockIdx.z * kTN;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gid = lane >> 2, t4 = lane & 3;
-
-  // per-thread share of one K chunk
-  constexpr int kAVec = OUT_BF16 ? (kTM * kTK / 8) / 128 : (kTM * kTK / 4) / 128;  // 4 or 8
-  constexpr int kWVec = (kTK * kTN / 8) / 128;                                      // 4
-  uint4 ra[kAVec], rw[kWVec];
-
-  auto load_chunk = [&](int k0) {
-#pragma unroll
-    for (int i = 0; i < kAVec; ++i) {
-      const int idx = tid + 128 * i;
-      const int row = OUT_BF16 ? idx / 8 : idx / 16;
-      const int col = OUT_BF16 ? 8 * (idx % 8) : 4 * (idx % 16);
-      const int b = m0 + row;
-      ra[i] = make_uint4(0, 0, 0, 0);
-      if (b < B) {
-        const int64_t off = (int64_t)b * o_sb + (int64_t)h * o_sh + k0 + col;
-        ra[i] = OUT_BF16 ? *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(outp) + off)
-                         : *reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(outp) + off);
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    // One SM's bulk copies from a single issuing thread complete one after
+    // another, so the boxes of a stage go out from different lanes: box i
+    // (W tiles, then the out tile) of stage s from lane nbox * s + i (the
+    // launcher keeps nbox * stages <= 32).
+    const int nbox = 2 * p.mh + 1;
+    if (lane == 0) {
+      tma_prefetch(&wmap);
+      tma_prefetch(&omap);
+    }
+    int issued = 0;
+    for (int k = 0; k < kKChunks; ++k) {
+      const int s = k % R;
+      int ok = 1;
+      if (lane == 0) {
+        if (k >= R) ok = wait(raw_empty(s), ((k / R) - 1) & 1, abort_flag);
+        if (ok) mbar_arrive_expect_tx(raw_full(s), p.tx_bytes);
       }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const int i = lane - nbox * s;
+      if (i >= 0 && i < nbox) {
+        const uint32_t st = sbase + (uint32_t)s * p.raw_bytes;
+        if (i < 2 * p.mh)
+          tma_load_3d(st + (uint32_t)i * kWBox, &wmap, 64 * i, kKC * k, h, raw_full(s));
+        else
+          tma_load_3d(st + (uint32_t)(2 * p.mh) * kWBox, &omap, kKC * k, h, b0, raw_full(s));
+      }
+      issued = k + 1;
     }
-#pragma unroll
-    for (int i = 0; i < kWVec; ++i) {
-      const int idx = tid + 128 * i;
-      const int kr = idx / 8, n = n0 + 8 * (idx % 8);
-      rw[i] = make_uint4(0, 0, 0, 0);
-      if (n < Dv)
-        rw[i] = *reinterpret_cast<const uint4*>(W + (int64_t)h * w_sh + (int64_t)(k0 + kr) * w_sj + n);
-    }
-  };
-  auto store_chunk = [&]() {
-#pragma unroll
-    for (int i = 0; i < kAVec; ++i) {
-      const int idx = tid + 128 * i;
-      if (OUT_BF16) {
-        *reinterpret_cast<uint4*>(&a_hi[idx / 8][8 * (idx % 8)]) = ra[i];
-      } else {
-        const int row = idx / 16, col = 4 * (idx % 16);
-        const float f[4] = {__uint_as_float(ra[i].x), __uint_as_float(ra[i].y),
-                            __uint_as_float(ra[i].z), __uint_as_float(ra[i].w)};
-        uint32_t hi[2], lo[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(f[2 * e]), h1 = __float2bfloat16_rn(f[2 * e + 1]);
-          hi[e] = pack_bf16(h0, h1);
-          lo[e] = pack_bf16(__float2bfloat16_rn(f[2 * e] - __bfloat162float(h0)),
-                            __float2bfloat16_rn(f[2 * e + 1] - __bfloat162float(h1)));
+    // copies still in flight after an abort land before the CTA exits
+    if (lane == 0)
+      for (int k = issued - R < 0 ? 0 : issued - R; k < issued && *abort_flag; ++k) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(raw_full(k % R), (k / R) & 1) && clock64() - t0 < kTimeoutCycles) {
         }
-        *reinterpret_cast<uint2*>(&a_hi[row][col]) = make_uint2(hi[0], hi[1]);
-        *reinterpret_cast<uint2*>(&a_lo[row][col]) = make_uint2(lo[0], lo[1]);
       }
-    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, p.nt, true, false);
+      bool ok = true;
+      for (int k = 0; k < kKChunks && ok; ++k) {
+        const int s = k % R, c = k % kConvStages;
+        ok = wait(raw_full(s), (k / R) & 1, abort_flag);
+        if (ok && !p.out_bf16) ok = wait(conv_full(c), (k / kConvStages) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t st = sbase + (uint32_t)s * p.raw_bytes;
+        // out^T operands: K-major [nt rows][64 j]; f32 out gives hi and lo
+        const uint32_t o0 = p.out_bf16 ? st + (uint32_t)(2 * p.mh) * kWBox
+                                       : sbase + p.off_conv + (uint32_t)c * 2 * p.o_bytes;
+        const int nterms = p.out_bf16 ? 1 : 2;
+        for (int m = 0; m < p.mh; ++m) {
+          const uint64_t a0 = sw128_desc(st + (uint32_t)(2 * m) * kWBox, kWBox, 1024);
+          for (int t = 0; t < nterms; ++t) {
+            const uint64_t bd = sw128_desc(o0 + (uint32_t)t * p.o_bytes, 16, 1024);
 #pragma unroll
-    for (int i = 0; i < kWVec; ++i) {
-      const int idx = tid + 128 * i;
-      *reinterpret_cast<uint4*>(&w_s[idx / 8][8 * (idx % 8)]) = rw[i];
-    }
-  };
-
-  float acc[8][4];
-#pragma unroll
-  for (int n = 0; n < 8; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
-
-  load_chunk(0);
-  for (int k0 = 0; k0 < kLatent; k0 += kTK) {
-    __syncthreads();  // previous chunk's fragments are read
-    store_chunk();
-    __syncthreads();
-    if (k0 + kTK < kLatent) load_chunk(k0 + kTK);  // in flight during the MMAs below
-#pragma unroll
-    for (int kk = 0; kk < kTK; kk += 16) {
-      const int ar = 16 * warp + (lane & 15), ac = kk + 8 * (lane >> 4);
-      uint32_t ah[4], al[4];
-      ldsm_x4(smem_u32(&a_hi[ar][ac]), ah[0], ah[1], ah[2], ah[3]);
-      if (!OUT_BF16) ldsm_x4(smem_u32(&a_lo[ar][ac]), al[0], al[1], al[2], al[3]);
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {  // two n-tiles of 8 per ldmatrix
-        const int wr = kk + (lane & 7) + 8 * ((lane >> 3) & 1), wc = 16 * np + 8 * (lane >> 4);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(smem_u32(&w_s[wr][wc]), b0, b1, b2, b3);
-        mma_bf16_16816(acc[2 * np], ah, b0, b1);
-        mma_bf16_16816(acc[2 * np + 1], ah, b2, b3);
-        if (!OUT_BF16) {
-          mma_bf16_16816(acc[2 * np], al, b0, b1);
-          mma_bf16_16816(acc[2 * np + 1], al, b2, b3);
+            for (int kk = 0; kk < 4; ++kk)  // K-steps of 16: A +2 KB (MN-major), B +32 B
+              mma_f16(tmem + 64 * m, a0 + (uint64_t)(kk * 128), bd + (uint64_t)(kk * 2), idesc,
+                      (k | kk | t) != 0);
+          }
+        }
+        mma_commit(raw_empty(s));
+        if (!p.out_bf16) mma_commit(conv_empty(c));
+      }
+      mma_commit(acc_full);
+      if (!ok) {  // let issued MMAs finish before the accumulators are freed
+        const long long t0 = clock64();
+        while (!mbar_try_wait(acc_full, 0) && clock64() - t0 < kTimeoutCycles) {
         }
       }
     }
-  }
-  const int r0 = m0 + 16 * warp + gid;
+  } else {
+    // ---------------------------------------------------------------- converters + epilogue
+    const int ct = threadIdx.x - 64;  // 0..127
+    bool ok = true;
+    if (!p.out_bf16) {
+      const int items = p.nt * 8;  // (row, 8-column group) per chunk
+      for (int k = 0; k < kKChunks && ok; ++k) {
+        const int s = k % R, c = k % kConvStages;
+        ok = wait(raw_full(s), (k / R) & 1, abort_flag);
+        if (ok && k >= kConvStages) ok = wait(conv_empty(c), ((k / kConvStages) - 1) & 1, abort_flag);
+        if (!ok) break;
+        const uint8_t* stage = smem + (size_t)s * p.raw_bytes + (size_t)(2 * p.mh) * kWBox;
+        const uint32_t hi = sbase + p.off_conv + (uint32_t)c * 2 * p.o_bytes;
+        const uint32_t lo = hi + p.o_bytes;
+        for (int i = ct; i < items; i += 128) {
+          const int r = i >> 3, g = i & 7;
+          const float4 x0 = *reinterpret_cast<const float4*>(stage + r * 256 + g * 32);
+          const float4 x1 = *reinterpret_cast<const float4*>(stage + r * 256 + g * 32 + 16);
+          const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          uint32_t ph[4], pl[4];
 #pragma unroll
-  for (int n = 0; n < 8; ++n) {
-    const int c = n0 + 8 * n + 2 * t4;
-    if (c >= Dv) continue;
-    if (r0 < B)
-      *reinterpret_cast<float2*>(y + (int64_t)r0 * y_sb + (int64_t)h * y_sh + c) =
-          make_float2(acc[n][0], acc[n][1]);
-    if (r0 + 8 < B)
-      *reinterpret_cast<float2*>(y + (int64_t)(r0 + 8) * y_sb + (int64_t)h * y_sh + c) =
-          make_float2(acc[n][2], acc[n][3]);
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t h0 = bf16_bits(v[2 * e]), h1 = bf16_bits(v[2 * e + 1]);
+            const float r0 = v[2 * e] - __uint_as_float(h0 << 16);
+            const float r1 = v[2 * e + 1] - __uint_as_float(h1 << 16);
+            ph[e] = h0 | (h1 << 16);
+            pl[e] = bf16_bits(r0) | (bf16_bits(r1) << 16);
+          }
+          const uint32_t off = (uint32_t)r * 128 + ((uint32_t)(g ^ (r & 7)) << 4);
+          st_shared_v4(hi + off, ph[0], ph[1], ph[2], ph[3]);
+          st_shared_v4(lo + off, pl[0], pl[1], pl[2], pl[3]);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(conv_full(c));
+      }
+    }
+    if (ok) ok = wait(acc_full, 0, abort_flag) && !*abort_flag;
+    if (ok) {
+      tc_fence_after();
+      const int q = warp & 3;  // TMEM lanes 32q .. 32q + 31
+      for (int m = 0; m < p.mh; ++m) {
+        const int v = 128 * m + 32 * q + lane;
+        for (int c0 = 0; c0 < p.nt; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 64 * m + c0, r);
+          tmem_wait_ld();
+          if (v < p.Dv) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int b = b0 + c0 + i;
+              if (c0 + i < p.nt && b < p.B)
+                p.y[(int64_t)b * p.y_sb + (int64_t)h * p.y_sh + v] = __uint_as_float(r[i]);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(p.mh == 2 ? 128u : 64u)
+                 : "memory");
   }
 }
 
-template <int NT>
-cudaError_t launch_nt(const void* o, int out_bf16, int64_t o_sb, int64_t o_sh,
-                      const __nv_bfloat16* W, int64_t w_sh, int64_t w_sj, float* y,
-                      int64_t y_sb, int64_t y_sh, int B, int H, cudaStream_t stream) {
-  dim3 grid((B + kMTile - 1) / kMTile, H);
-  if (out_bf16)
-    vup_kernel<NT, true><<<grid, kWarps * 32, 0, stream>>>(o, o_sb, o_sh, W, w_sh, w_sj, y,
-                                                           y_sb, y_sh, B);
-  else
-    vup_kernel<NT, false><<<grid, kWarps * 32, 0, stream>>>(o, o_sb, o_sh, W, w_sh, w_sj, y,
-                                                            y_sb, y_sh, B);
+std::mutex g_vup_mu;
+bool g_vup_attr[64] = {};
+
+}  // namespace
+
+bool vup_supported(const void* out_latent, int out_bf16, int64_t o_sb, int64_t o_sh,
+                   const void* W, int64_t w_sh, int64_t w_sj) {
+  const int64_t esz = out_bf16 ? 2 : 4;
+  auto a16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; };
+  return a16(out_latent) && a16(W) && (o_sb * esz) % 16 == 0 && (o_sh * esz) % 16 == 0 &&
+         (w_sh * 2) % 16 == 0 && (w_sj * 2) % 16 == 0;
+}
+
+cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64_t o_sh,
+                       const void* W, int64_t w_sh, int64_t w_sj, float* y, int64_t y_sb,
+                       int64_t y_sh, int B, int H, int Dv, cudaStream_t stream) {
+  if (B == 0 || H == 0 || Dv == 0) return cudaSuccess;
+  if (!vup_supported(out_latent, out_bf16, o_sb, o_sh, W, w_sh, w_sj) || Dv > 256 || Dv % 16)
+    return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!sm100_device(dev)) return cudaErrorNotSupported;
+  auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
+  if (!encode) return cudaErrorNotSupported;
+
+  VupParams p{};
+  p.y = y;
+  p.y_sb = y_sb;
+  p.y_sh = y_sh;
+  p.B = B;
+  p.H = H;
+  p.Dv = Dv;
+  p.mh = Dv > 128 ? 2 : 1;
+  p.nt = B >= kMaxN ? kMaxN : ((B + 15) / 16) * 16;
+  p.out_bf16 = out_bf16;
+  p.o_bytes = (uint32_t)p.nt * (out_bf16 ? 128u : 256u);
+  const uint32_t conv_tile = (uint32_t)p.nt * 128u;  // one bf16 K-major tile
+  p.tx_bytes = (uint32_t)(2 * p.mh) * kWBox + p.o_bytes;
+  p.raw_bytes = (p.tx_bytes + 1023u) & ~1023u;
+  const uint32_t conv_bytes = out_bf16 ? 0u : ((kConvStages * 2 * conv_tile + 1023u) & ~1023u);
+  int R = (int)((kSmemBudget - conv_bytes) / p.raw_bytes);
+  p.raw_stages = R > kMaxRaw ? kMaxRaw : R;
+  while (p.raw_stages * (2 * p.mh + 1) > 32) --p.raw_stages;  // one issuing lane per box
+  p.off_conv = (uint32_t)p.raw_stages * p.raw_bytes;
+  p.o_bytes = out_bf16 ? p.o_bytes : conv_tile;  // the MMA reads hi/lo tiles of nt x 128 B
+  p.off_bar = p.off_conv + conv_bytes;
+  const uint32_t smem = p.off_bar + 8 * (2 * kMaxRaw + 2 * kConvStages + 1) + 16 + 1024;
+
+  // W as [H][512][Dv] (v innermost): boxes of 64 v x 64 j, MN-major for the MMA
+  CUtensorMap wmap, omap;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)Dv, (cuuint64_t)kLatent, (cuuint64_t)H};
+    cuuint64_t strides[2] = {(cuuint64_t)w_sj * 2, (cuuint64_t)w_sh * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)kKC, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(W), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  // out as [B][H][512] (j innermost): boxes of 64 j x 1 head x nt requests
+  {
+    const uint64_t esz = out_bf16 ? 2 : 4;
+    cuuint64_t dims[3] = {(cuuint64_t)kLatent, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)o_sh * esz, (cuuint64_t)o_sb * esz};
+    cuuint32_t box[3] = {(cuuint32_t)kKC, 1, (cuuint32_t)p.nt};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (encode(&omap,
+               out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+               const_cast<void*>(out_latent), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE,
+               out_bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_vup_mu);
+    if (!g_vup_attr[dev & 63]) {
+      cudaError_t e = cudaFuncSetAttribute(vup_sm100_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kSmemBudget + 4096);
+      if (e != cudaSuccess) return e;
+      g_vup_attr[dev & 63] = true;
+    }
+  }
+  dim3 grid(H, (B + p.nt - 1) / p.nt);
+  vup_sm100_kernel<<<grid, kThreads, smem, stream>>>(wmap, omap, p);
   count_launch();
   return cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64_t o_sh,
-                       const void* W, int64_t w_sh, int64_t w_sj, float* y,
-                       int64_t y_sb, int64_t y_sh, int B, int H, int Dv,
-                       cudaStream_t stream) {
-  if (B == 0 || H == 0 || Dv == 0) return cudaSuccess;
-  const __nv_bfloat16* w = reinterpret_cast<const __nv_bfloat16*>(W);
-  const int ovec = out_bf16 ? 8 : 4;  // elements per 16 bytes
-  const bool tiled = (reinterpret_cast<uintptr_t>(out_latent) & 15u) == 0 &&
-                     (reinterpret_cast<uintptr_t>(W) & 15u) == 0 &&
-                     (reinterpret_cast<uintptr_t>(y) & 7u) == 0 && o_sb % ovec == 0 &&
-                     o_sh % ovec == 0 && w_sh % 8 == 0 && w_sj % 8 == 0 && y_sb % 2 == 0 &&
-                     y_sh % 2 == 0;
-  if (tiled) {
-    dim3 grid((B + kTM - 1) / kTM, H, (Dv + kTN - 1) / kTN);
-    if (out_bf16)
-      vup_tiled_kernel<true><<<grid, 128, 0, stream>>>(out_latent, o_sb, o_sh, w, w_sh, w_sj, y,
-                                                       y_sb, y_sh, B, Dv);
-    else
-      vup_tiled_kernel<false><<<grid, 128, 0, stream>>>(out_latent, o_sb, o_sh, w, w_sh, w_sj, y,
-                                                        y_sb, y_sh, B, Dv);
-    count_launch();
-    return cudaGetLastError();
+cudaError_t status_read_clear_vup(int* code) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_vup_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (v != 0) {
+    int zero = 0;
+    e = cudaMemcpyToSymbol(g_vup_status, &zero, sizeof(int));
   }
-  switch (Dv) {
-#define TPLA_VUP_CASE(D) \
-  case D: return launch_nt<D / 8>(out_latent, out_bf16, o_sb, o_sh, w, w_sh, w_sj, y, y_sb, y_sh, B, H, stream);
-    TPLA_VUP_CASE(16) TPLA_VUP_CASE(32) TPLA_VUP_CASE(48) TPLA_VUP_CASE(64)
-    TPLA_VUP_CASE(80) TPLA_VUP_CASE(96) TPLA_VUP_CASE(112) TPLA_VUP_CASE(128)
-    TPLA_VUP_CASE(144) TPLA_VUP_CASE(160) TPLA_VUP_CASE(176) TPLA_VUP_CASE(192)
-    TPLA_VUP_CASE(208) TPLA_VUP_CASE(224) TPLA_VUP_CASE(240) TPLA_VUP_CASE(256)
-#undef TPLA_VUP_CASE
-    default: return cudaErrorInvalidValue;
-  }
+  *code = v;
+  return e;
 }
 
 }  // namespace tpla

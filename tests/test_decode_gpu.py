@@ -47,7 +47,7 @@ RAGGED = [1, 63, 64, 65, 300, 0, 129]
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
-@pytest.mark.parametrize("H", [16, 64, 128])
+@pytest.mark.parametrize("H", [16, 64, 128, 256])
 @pytest.mark.parametrize("G,rope", [(1, "replicate"), (2, "replicate"), (2, "split"),
                                     (4, "replicate"), (4, "split"), (8, "replicate")])
 def test_ragged_paged(cuda_dev, kernel, H, G, rope):
@@ -206,3 +206,20 @@ def test_hadamard_tpla_g2_matches_oracle_on_rotated_inputs(cuda_dev):
                                np.float32(w.scale))
     assert_out_close(to_np(out), ro)
     assert_lse_close(to_np(lse), rl)
+
+
+def test_auto_never_falls_back_to_the_portable_kernel(cuda_dev):
+    """G = 8 is outside the tcgen05 kernel: the automatic choice reports
+    UNSUPPORTED before any launch instead of running another kernel; the
+    portable kernel runs it when named."""
+    w = make_inputs(2, 16, [300, 64], paged=True, decay=True, seed=131)
+    d = to_device(w, cuda_dev)
+    before = tp.launch_count()
+    with pytest.raises(tp.TplaError) as e:
+        tp.decode(d["q"], d["cache"], d["seq_lens"], d["page_table"], 8, "replicate", w.scale)
+    assert e.value.status == -2
+    assert tp.launch_count() == before
+    out, lse = run(cuda_dev, w, 8, "replicate", "generic", d=d)
+    ro, rl = oracle_decode(w, 8, "replicate")
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
