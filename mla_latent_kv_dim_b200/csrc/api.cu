@@ -402,6 +402,7 @@ int tpla_rotate_apply(tpla_tensor* buf, const tpla_tensor* U, void* scratch,
   int64_t chunk = (int64_t)(scratch_bytes / per_b);
   if (chunk > B) chunk = B;
   if (chunk > (1 << 24)) chunk = 1 << 24;
+  if (chunk * H > (1LL << 30)) chunk = (1LL << 30) / H;  // store grid stays below 2^31 blocks
   cudaError_t e = launch_rotate(buf->data, B, H, sb, sh, U->data, reinterpret_cast<float*>(scratch),
                                 chunk, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
