@@ -12,7 +12,7 @@ The Walsh-Hadamard reparameterisation is applied once to q, the cache and
 Metric: latent-KV GB/s = algorithmic cache bytes per step / step time
 (also decode tokens/s per layer).  Inputs (2.4 GB) exceed the 126 MB L2, so
 no flush is needed between steps.  Multi-GPU runs are independent replicas
-(the path has no cross-GPU exchange on one node in this build).
+(the decode path has no cross-GPU exchange).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """

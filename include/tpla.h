@@ -60,7 +60,7 @@ enum tpla_dtype { TPLA_BF16 = 1, TPLA_F32 = 2, TPLA_I32 = 3 };
 enum tpla_status {
   TPLA_OK = 0,
   TPLA_ERR_INVALID_ARG = -1,   /* null pointer, shape/stride/dtype mismatch  */
-  TPLA_ERR_UNSUPPORTED = -2,   /* valid request this build cannot run        */
+  TPLA_ERR_UNSUPPORTED = -2,   /* valid request the library cannot run       */
   TPLA_ERR_CUDA = -3,          /* a CUDA call failed; see tpla_last_cuda_error */
   TPLA_ERR_WORKSPACE = -4,     /* workspace missing or too small             */
   TPLA_ERR_DEVICE_TIMEOUT = -5,/* a kernel gave up waiting (device status)   */

@@ -412,7 +412,7 @@ const char* tpla_error_string(int status) {
   switch (status) {
     case TPLA_OK: return "ok";
     case TPLA_ERR_INVALID_ARG: return "invalid argument";
-    case TPLA_ERR_UNSUPPORTED: return "unsupported by this build";
+    case TPLA_ERR_UNSUPPORTED: return "unsupported by the library";
     case TPLA_ERR_CUDA: return "CUDA error";
     case TPLA_ERR_WORKSPACE: return "workspace missing or too small";
     case TPLA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
