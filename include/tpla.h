@@ -250,6 +250,41 @@ TPLA_API int tpla_hadamard_apply(tpla_tensor* buf, int dim, tpla_stream_t stream
 TPLA_API int tpla_vup_combine(const tpla_tensor* out_latent, const tpla_tensor* W_uv,
                      tpla_tensor* y, tpla_stream_t stream);
 
+/*
+ * PCA reparameterisation (TPLA abstract; feature request, "Directions under
+ * investigation": PCA beside the Hadamard transform as the orthogonal change
+ * of basis applied before slicing; the TPLA review's referee comments on
+ * Sec. 4.3.2 / Eq. 25: PCA of the latent cache features, rope excluded).
+ * The library computes the calibration statistics and applies a basis; the
+ * 512 x 512 eigensolve that turns the covariance into U is the caller's,
+ * offline.
+ *
+ * tpla_latent_covariance -- accumulates, over the first 512 columns x of every
+ * row of `rows` ([N, >= 512] or [B, H, >= 512] bf16, innermost contiguous,
+ * 16-byte aligned rows):  C[i][j] += sum x_i x_j  and  s[i] += sum x_i.
+ *   C [512, 512] f32 and s [512] f32, zeroed by the caller before the first
+ *   call; several calls accumulate.  f32 arithmetic, atomic adds (the sum
+ *   order is not fixed).
+ * tpla_covariance_finalize -- mean = s / n, cov = C / n - mean mean^T
+ *   (n = rows accumulated), both f32; cov [512, 512], mean [512].
+ * tpla_rotate_apply -- in place, x <- x U on the first 512 columns of every row
+ *   of `buf` (same layouts as `rows` above); other columns untouched.
+ *   U [512, 512] bf16, row-major and contiguous (U[j][n] multiplies x_j into
+ *   output n).  `scratch` is caller device memory of at least
+ *   H * 512 * 4 bytes (H = 1 for two-dimensional buf); larger scratch lets
+ *   the rows go through in fewer, longer passes.  Tensor-core bf16 products,
+ *   f32 accumulation, one bf16 rounding on store.
+ * Errors: TPLA_ERR_INVALID_ARG for shapes, dtypes, strides or alignment;
+ * TPLA_ERR_WORKSPACE for missing or short scratch.
+ */
+TPLA_API int tpla_latent_covariance(const tpla_tensor* rows, tpla_tensor* C, tpla_tensor* s,
+                                    tpla_stream_t stream);
+TPLA_API int tpla_covariance_finalize(const tpla_tensor* C, const tpla_tensor* s, int64_t n,
+                                      tpla_tensor* cov, tpla_tensor* mean,
+                                      tpla_stream_t stream);
+TPLA_API int tpla_rotate_apply(tpla_tensor* buf, const tpla_tensor* U, void* scratch,
+                               size_t scratch_bytes, tpla_stream_t stream);
+
 /* Human-readable name of a tpla_status code (static string). */
 TPLA_API const char* tpla_error_string(int status);
 

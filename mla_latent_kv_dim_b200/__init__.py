@@ -6,10 +6,10 @@ CUDA kernels for sm_100a.  This package holds the ctypes binding
 workloads (``workloads``).
 """
 from ._native import (TplaError, decode, decode_simple, decode_workspace_size,  # noqa: F401
-                      device_status, error_string, hadamard_apply, launch_count, lse_merge, lib,
-                      selftest_wait_timeout,
+                      device_status, error_string, hadamard_apply, latent_covariance,
+                      launch_count, lse_merge, lib, rotate_apply, selftest_wait_timeout,
                       version, vup_combine)
 
 __all__ = ["TplaError", "decode", "decode_simple", "decode_workspace_size", "device_status",
-           "selftest_wait_timeout",
+           "selftest_wait_timeout", "latent_covariance", "rotate_apply",
            "error_string", "hadamard_apply", "launch_count", "lse_merge", "lib", "version", "vup_combine"]

@@ -76,10 +76,15 @@ def lib() -> ctypes.CDLL:
             L.tpla_error_string.restype = ctypes.c_char_p
             L.tpla_get_device_status.argtypes = [ctypes.c_void_p, _P(ctypes.c_int)]
             L.tpla_selftest_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_void_p]
+            L.tpla_latent_covariance.argtypes = [T, T, T, ctypes.c_void_p]
+            L.tpla_covariance_finalize.argtypes = [T, T, ctypes.c_int64, T, T, ctypes.c_void_p]
+            L.tpla_rotate_apply.argtypes = [T, T, ctypes.c_void_p, ctypes.c_size_t,
+                                            ctypes.c_void_p]
             for f in ("tpla_decode_ex", "tpla_decode", "tpla_decode_workspace_size",
                       "tpla_lse_merge", "tpla_hadamard_apply", "tpla_vup_combine",
                       "tpla_last_cuda_error", "tpla_get_device_status", "tpla_version",
-                      "tpla_selftest_wait_timeout"):
+                      "tpla_selftest_wait_timeout", "tpla_latent_covariance",
+                      "tpla_covariance_finalize", "tpla_rotate_apply"):
                 getattr(L, f).restype = ctypes.c_int
             L.tpla_launch_count.restype = ctypes.c_int64
             _lib = L
@@ -239,6 +244,42 @@ def vup_combine(out_latent, W_uv, y=None, stream=None):
                                 _stream(stream))
     _check("tpla_vup_combine", rc)
     return y
+
+
+def latent_covariance(rows, stream=None):
+    """(mean [512], covariance [512, 512]) f32 of the first 512 columns of
+    the calibration rows ([N, >= 512] or [B, H, >= 512] bf16), computed by
+    tpla_latent_covariance + tpla_covariance_finalize."""
+    _on_current_device(rows)
+    dev = rows.device
+    C = torch.zeros((512, 512), dtype=torch.float32, device=dev)
+    ssum = torch.zeros((512,), dtype=torch.float32, device=dev)
+    st = _stream(stream)
+    _check("tpla_latent_covariance",
+           lib().tpla_latent_covariance(_ref(desc(rows)), _ref(desc(C)), _ref(desc(ssum)), st))
+    n = rows.shape[0] * (rows.shape[1] if rows.dim() == 3 else 1)
+    cov = torch.empty_like(C)
+    mean = torch.empty_like(ssum)
+    _check("tpla_covariance_finalize",
+           lib().tpla_covariance_finalize(_ref(desc(C)), _ref(desc(ssum)), int(n),
+                                          _ref(desc(cov)), _ref(desc(mean)), st))
+    return mean, cov
+
+
+def rotate_apply(buf, U, scratch=None, stream=None):
+    """In place x <- x U on the first 512 columns of every row of ``buf``
+    (bf16), U [512, 512] bf16 (tpla_rotate_apply).  ``scratch`` (a device
+    tensor of at least H * 512 f32) is allocated when not given."""
+    _on_current_device(buf, U, scratch)
+    if scratch is None:
+        lead = buf.shape[0]
+        per = (buf.shape[1] if buf.dim() == 3 else 1) * 512
+        scratch = torch.empty((max(1, min(lead, max(1, (1 << 24) // per))) * per,),
+                              dtype=torch.float32, device=buf.device)
+    rc = lib().tpla_rotate_apply(_ref(desc(buf)), _ref(desc(U)), scratch.data_ptr(),
+                                 scratch.numel() * scratch.element_size(), _stream(stream))
+    _check("tpla_rotate_apply", rc)
+    return buf
 
 
 def device_status(stream=None) -> int:

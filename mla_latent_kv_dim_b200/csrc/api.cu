@@ -333,6 +333,76 @@ int tpla_vup_combine(const tpla_tensor* out_latent, const tpla_tensor* W_uv, tpl
   return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
 }
 
+namespace {
+// [N, >= 512] or [B, H, >= 512] bf16 rows, innermost contiguous, 16-byte rows.
+bool latent_rows(const tpla_tensor* t, int64_t* B, int64_t* H, int64_t* sb, int64_t* sh) {
+  if (!t || t->dtype != TPLA_BF16 || (t->ndim != 2 && t->ndim != 3)) return false;
+  if (!check_tensor(t, TPLA_BF16, t->ndim) || t->shape[t->ndim - 1] < kLatent) return false;
+  if (t->ndim == 2) {
+    *B = t->shape[0];
+    *H = 1;
+    *sb = t->stride[0];
+    *sh = 0;
+  } else {
+    *B = t->shape[0];
+    *H = t->shape[1];
+    *sb = t->stride[0];
+    *sh = t->stride[1];
+  }
+  if (*B * *H > 0 && (!aligned16(t->data) || *sb % 8 || *sh % 8)) return false;
+  return true;
+}
+}  // namespace
+
+int tpla_latent_covariance(const tpla_tensor* rows, tpla_tensor* C, tpla_tensor* s,
+                           tpla_stream_t stream) {
+  int64_t B, H, sb, sh;
+  if (!latent_rows(rows, &B, &H, &sb, &sh)) return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(C, TPLA_F32, 2) || C->shape[0] != kLatent || C->shape[1] != kLatent ||
+      !check_tensor(s, TPLA_F32, 1) || s->shape[0] != kLatent)
+    return TPLA_ERR_INVALID_ARG;
+  if (B * H > (int64_t)65535 * 2048 || H > (1 << 30)) return TPLA_ERR_UNSUPPORTED;
+  cudaError_t e = launch_latent_stats(rows->data, B, H, sb, sh, reinterpret_cast<float*>(C->data),
+                                      C->stride[0], reinterpret_cast<float*>(s->data),
+                                      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
+}
+
+int tpla_covariance_finalize(const tpla_tensor* C, const tpla_tensor* s, int64_t n,
+                             tpla_tensor* cov, tpla_tensor* mean, tpla_stream_t stream) {
+  if (n <= 0) return TPLA_ERR_INVALID_ARG;
+  for (const tpla_tensor* m : {C, static_cast<const tpla_tensor*>(cov)})
+    if (!check_tensor(m, TPLA_F32, 2) || m->shape[0] != kLatent || m->shape[1] != kLatent)
+      return TPLA_ERR_INVALID_ARG;
+  for (const tpla_tensor* v : {s, static_cast<const tpla_tensor*>(mean)})
+    if (!check_tensor(v, TPLA_F32, 1) || v->shape[0] != kLatent) return TPLA_ERR_INVALID_ARG;
+  cudaError_t e = launch_covariance_finalize(
+      reinterpret_cast<const float*>(C->data), C->stride[0],
+      reinterpret_cast<const float*>(s->data), n, reinterpret_cast<float*>(cov->data),
+      cov->stride[0], reinterpret_cast<float*>(mean->data), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
+}
+
+int tpla_rotate_apply(tpla_tensor* buf, const tpla_tensor* U, void* scratch,
+                      size_t scratch_bytes, tpla_stream_t stream) {
+  int64_t B, H, sb, sh;
+  if (!latent_rows(buf, &B, &H, &sb, &sh)) return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(U, TPLA_BF16, 2) || U->shape[0] != kLatent || U->shape[1] != kLatent ||
+      U->stride[0] != kLatent || !aligned16(U->data))
+    return TPLA_ERR_INVALID_ARG;
+  if (B * H == 0) return TPLA_OK;
+  if (H > 65535 || B > (1LL << 31) - 1) return TPLA_ERR_UNSUPPORTED;
+  const size_t per_b = (size_t)H * kLatent * sizeof(float);
+  if (!scratch || !aligned16(scratch) || scratch_bytes < per_b) return TPLA_ERR_WORKSPACE;
+  int64_t chunk = (int64_t)(scratch_bytes / per_b);
+  if (chunk > B) chunk = B;
+  if (chunk > (1 << 24)) chunk = 1 << 24;
+  if (chunk * H > (1LL << 30)) chunk = (1LL << 30) / H;  // store grid stays below 2^31 blocks
+  cudaError_t e = launch_rotate(buf->data, B, H, sb, sh, U->data, reinterpret_cast<float*>(scratch),
+                                chunk, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
+}
+
 const char* tpla_error_string(int status) {
   switch (status) {
     case TPLA_OK: return "ok";

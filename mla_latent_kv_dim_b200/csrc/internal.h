@@ -82,6 +82,17 @@ cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64
                        int64_t y_sb, int64_t y_sh, int B, int H, int Dv,
                        cudaStream_t stream);
 
+// ---------------------------------------------------------------- PCA reparameterisation
+// Rows are the first 512 columns of a [B, H, >= 512] bf16 view (element
+// strides sb, sh; innermost contiguous).
+cudaError_t launch_latent_stats(const void* x, int64_t B, int64_t H, int64_t sb, int64_t sh,
+                                float* C, int64_t c_s0, float* s, cudaStream_t stream);
+cudaError_t launch_covariance_finalize(const float* C, int64_t c_s0, const float* s, int64_t n,
+                                       float* cov, int64_t v_s0, float* mean,
+                                       cudaStream_t stream);
+cudaError_t launch_rotate(void* x, int64_t B, int64_t H, int64_t sb, int64_t sh, const void* U,
+                          float* scratch, int64_t chunk_b, cudaStream_t stream);
+
 // ---------------------------------------------------------------- launch counter
 // Called once per kernel launch by every launcher.
 void count_launch(int n = 1);

@@ -52,6 +52,12 @@ Readings taken where the pages are silent:
    each shard's share is taken the same way.  They are diagnostics: the
    deployed computation is the unscaled local softmax (reading 1), so no
    mu/nu factor enters it.
+10. The cache stores the latent after its RMS normalisation; the norm's
+   learned gain is absorbed into the up-projections (like the rotation U,
+   [REVIEW pith_extraction.key_machinery]), so a stored row is x / rms(x),
+   taken over each of ``norm_groups`` contiguous shards (one group: exact
+   MLA; G groups: every TPLA rank normalises its own slice).  The rotation,
+   when used, comes first; eps is added to the mean square.
 """
 
 from __future__ import annotations
@@ -427,6 +433,66 @@ def fold_vup_ref(W_uv, U):
     """V-up weights for outputs in the rotated space: W'[h] = U^T W[h], so
     that (out U) W' = out W (the rotation absorbed into the projection)."""
     return np.einsum("ji,hjk->hik", np.asarray(U, np.float64), np.asarray(W_uv, np.float64))
+
+
+# ---------------------------------------------------------------------------
+# Cache append: the latent of a new token, normalised per shard and stored
+# ---------------------------------------------------------------------------
+
+def rms_norm_groups_ref(x, groups, eps):
+    """RMS normalisation of each of ``groups`` contiguous column blocks of the
+    rows of ``x`` (last axis): block / sqrt(mean(block^2) + eps) (reading 10).
+
+    [REVIEW pith_extraction.key_machinery]: Condition 1 asks the shards' RMS
+    norms to be proportional to the global norm, i.e. each device normalises
+    its own slice of the latent; ``groups = 1`` is the ordinary (global)
+    norm of exact MLA.
+    """
+    x = np.asarray(x, np.float64)
+    D = x.shape[-1]
+    if D % groups:
+        raise ValueError("groups must divide the row width")
+    d = D // groups
+    out = np.empty_like(x)
+    for g in range(groups):
+        blk = x[..., g * d:(g + 1) * d]
+        ms = (blk * blk).mean(axis=-1, keepdims=True)
+        out[..., g * d:(g + 1) * d] = blk / np.sqrt(ms + eps)
+    return out
+
+
+def cache_row_ref(kv_new, norm_groups, hadamard, eps):
+    """The stored cache row of a new token (reading 10).
+
+    ``kv_new`` [..., 576]: the token's latent before its normalisation
+    (columns 0..511) and its rope key (512..575, already position-encoded).
+    The latent is optionally rotated by the orthonormal Hadamard matrix
+    (the reparameterisation applied before slicing, [ISSUE] "Directions under
+    investigation"), then RMS-normalised over ``norm_groups`` contiguous
+    shards.  [REVIEW referee_report.significance]: Proposition 1, RMSNorm
+    commutes with an orthogonal transform, so with one group rotating before
+    or after the norm gives the same row.  The rope part is stored as given.
+    """
+    a = np.asarray(kv_new, np.float64)
+    x = a[..., :LATENT]
+    if hadamard:
+        x = x @ hadamard_matrix(LATENT)
+    return np.concatenate([rms_norm_groups_ref(x, norm_groups, eps), a[..., LATENT:]], axis=-1)
+
+
+def cache_append_ref(cache, kv_new, positions, page_table, norm_groups, hadamard, eps):
+    """A copy of ``cache`` with request b's new row stored at token
+    ``positions[b]``: paged, block ``page_table[b][pos // 64]`` row
+    ``pos % 64`` of [num_blocks, 64, 576]; contiguous (``page_table=None``),
+    row ``pos`` of [B, Lmax, 576].  Nothing else changes."""
+    out = np.array(cache, dtype=np.float64, copy=True)
+    rows = cache_row_ref(kv_new, norm_groups, hadamard, eps)
+    for b, pos in enumerate(np.asarray(positions).tolist()):
+        if page_table is None:
+            out[b, pos] = rows[b]
+        else:
+            out[np.asarray(page_table)[b][pos // BLOCK], pos % BLOCK] = rows[b]
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -255,3 +255,30 @@ def test_empty_batch_or_heads_is_a_no_op(B, H):
     assert _call(q, kv, seq, pt, 2, 0, out, lse) == 0
     assert _call(q, kv, seq, pt, 2, 0, out, lse, N._opts(0, None, "generic")) == 0
     assert tp.launch_count() == before
+
+
+def test_pca_entry_points_validate_without_launch():
+    L = tp.lib()
+    before = tp.launch_count()
+    B = ctypes.byref
+    rows = _fake((4, 64, 576), torch.bfloat16)
+    C = _fake((512, 512), torch.float32)
+    s = _fake((512,), torch.float32)
+    U = _fake((512, 512), torch.bfloat16)
+    # rows narrower than the latent, wrong dtype, misaligned
+    assert L.tpla_latent_covariance(B(_fake((4, 500), torch.bfloat16)), B(C), B(s), None) == -1
+    assert L.tpla_latent_covariance(B(_fake((4, 576), torch.float32)), B(C), B(s), None) == -1
+    bad = _fake((4, 576), torch.bfloat16, ptr=0x10002)
+    assert L.tpla_latent_covariance(B(bad), B(C), B(s), None) == -1
+    assert L.tpla_latent_covariance(B(rows), B(_fake((512, 256), torch.float32)), B(s), None) == -1
+    assert L.tpla_covariance_finalize(B(C), B(s), 0, B(C), B(s), None) == -1
+    # U must be [512, 512] bf16 row-major; scratch must hold one leading index
+    assert L.tpla_rotate_apply(B(rows), B(_fake((512, 256), torch.bfloat16)), 0x20000, 1 << 20,
+                               None) == -1
+    Ut = _fake((512, 512), torch.bfloat16)
+    Ut.stride[0], Ut.stride[1] = 1, 512
+    assert L.tpla_rotate_apply(B(rows), B(Ut), 0x20000, 1 << 20, None) == -1
+    assert L.tpla_rotate_apply(B(rows), B(U), None, 1 << 20, None) == -4
+    assert L.tpla_rotate_apply(B(rows), B(U), 0x20000, 64 * 512 * 4 - 16, None) == -4
+    assert L.tpla_rotate_apply(B(rows), B(U), 0x20008, 1 << 20, None) == -4
+    assert tp.launch_count() == before

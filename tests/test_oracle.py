@@ -535,3 +535,136 @@ def test_per_head_cosine_hand_computed():
     # symmetric, and invariant under positive scaling of either argument
     np.testing.assert_allclose(O.per_head_cosine(b, a), want, rtol=0, atol=1e-15)
     np.testing.assert_allclose(O.per_head_cosine(7.0 * a, 0.5 * b), want, rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Cache append: per-shard RMS normalisation (Condition 1 / Proposition 1)
+# ---------------------------------------------------------------------------
+
+def _cache_row_bruteforce(a, groups, hadamard, eps):
+    """Scalar-loop restatement on Python floats: Sylvester entries from the
+    popcount rule, sums of squares and square roots by hand."""
+    D = 512
+    x = [float(v) for v in a[:D]]
+    if hadamard:
+        y = []
+        for j in range(D):
+            acc = 0.0
+            for i in range(D):
+                sign = -1.0 if bin(i & j).count("1") % 2 else 1.0
+                acc += x[i] * sign
+            y.append(acc / math.sqrt(D))
+        x = y
+    d = D // groups
+    out = []
+    for g in range(groups):
+        blk = x[g * d:(g + 1) * d]
+        ms = sum(v * v for v in blk) / d
+        out += [v / math.sqrt(ms + eps) for v in blk]
+    return out + [float(v) for v in a[D:]]
+
+
+@pytest.mark.parametrize("groups,hadamard", [(1, False), (2, False), (4, True), (8, True)])
+def test_cache_row_matches_bruteforce(groups, hadamard):
+    a = np.random.default_rng(groups).standard_normal((2, 576)) * 3.0
+    got = O.cache_row_ref(a, groups, hadamard, 1e-6)
+    for b in range(2):
+        want = _cache_row_bruteforce(a[b], groups, hadamard, 1e-6)
+        np.testing.assert_allclose(got[b], want, rtol=1e-12, atol=1e-12)
+
+
+def test_proposition1_rmsnorm_commutes_with_hadamard():
+    """With one group, normalising then rotating equals rotating then
+    normalising: the orthogonal H keeps the RMS of a row."""
+    a = np.random.default_rng(3).standard_normal((5, 576)) * np.exp(-np.arange(576) / 128)
+    rot_first = O.cache_row_ref(a, 1, True, 1e-6)
+    norm_first = O.hadamard_ref(O.cache_row_ref(a, 1, False, 1e-6), 512)
+    np.testing.assert_allclose(rot_first, norm_first, rtol=0, atol=1e-12)
+    # with several groups it does not hold in general (the shards' energies differ)
+    g2 = O.hadamard_ref(O.cache_row_ref(a, 2, False, 1e-6), 512)
+    assert np.abs(O.cache_row_ref(a, 2, True, 1e-6) - g2).max() > 1e-3
+
+
+def test_condition1_spike_closed_forms():
+    """A latent concentrated on one channel: after the Hadamard rotation every
+    entry is +-1/sqrt(512), so every shard has the global RMS and the stored
+    row is the sign pattern for any number of groups (Condition 1 exact).
+    Without the rotation only the shard holding the channel is non-zero, at
+    sqrt(d) (d = 512 / groups), and the other shards stay 0."""
+    k, eps = 300, 0.0
+    a = np.zeros(576)
+    a[k] = 2.5
+    a[512:] = np.arange(64) * 0.5
+    H = O.hadamard_matrix(512)
+    for groups in (1, 2, 4, 8):
+        row = O.cache_row_ref(a, groups, True, eps)
+        np.testing.assert_allclose(row[:512], np.sign(H[k]), rtol=0, atol=1e-12)
+        np.testing.assert_array_equal(row[512:], a[512:])
+        d = 512 // groups
+        plain = O.cache_row_ref(a, groups, False, 1e-30)
+        want = np.zeros(512)
+        want[k] = math.sqrt(d)
+        np.testing.assert_allclose(plain[:512], want, rtol=1e-12, atol=1e-12)
+
+
+def test_cache_row_groups_have_unit_rms():
+    a = np.random.default_rng(4).standard_normal((3, 576)) * 0.01
+    eps = 1e-5
+    for groups in (1, 2, 4):
+        d = 512 // groups
+        x = O.hadamard_ref(a, 512)[:, :512]
+        row = O.cache_row_ref(a, groups, True, eps)
+        for g in range(groups):
+            ms = (x[:, g * d:(g + 1) * d] ** 2).mean(axis=1)
+            got = (row[:, g * d:(g + 1) * d] ** 2).mean(axis=1)
+            np.testing.assert_allclose(got, ms / (ms + eps), rtol=1e-12)
+
+
+def test_cache_append_placement_paged_and_contiguous():
+    rng = np.random.default_rng(5)
+    B, pages = 3, 3
+    cache = rng.standard_normal((8, 64, 576))
+    pt = np.array([[4, 1, 7], [0, 2, 3], [6, 5, 1]])
+    pos = np.array([130, 0, 63])
+    new = rng.standard_normal((B, 576))
+    got = O.cache_append_ref(cache, new, pos, pt, 2, True, 1e-6)
+    rows = O.cache_row_ref(new, 2, True, 1e-6)
+    want = cache.copy()
+    for b in range(B):
+        want[pt[b][pos[b] // 64], pos[b] % 64] = rows[b]
+    np.testing.assert_array_equal(got, want)
+    assert np.count_nonzero(np.any(got != cache, axis=-1)) == B  # nothing else changed
+    # the same rows land at the same tokens of a contiguous cache
+    contig = np.stack([cache[pt[b]].reshape(pages * 64, 576) for b in range(B)])
+    got_c = O.cache_append_ref(contig, new, pos, None, 2, True, 1e-6)
+    for b in range(B):
+        np.testing.assert_array_equal(got_c[b].reshape(pages, 64, 576), got[pt[b]])
+
+
+def test_cache_append_pins_catch_planted_mistakes(monkeypatch):
+    """Plant plausible mistakes in the oracle's normaliser; the brute-force
+    and closed-form pins must fail on each."""
+    good = O.rms_norm_groups_ref
+    a = np.random.default_rng(6).standard_normal(576)
+
+    def norm_over_width(x, groups, eps):  # one norm over all columns
+        return good(x, 1, eps)
+
+    def no_mean(x, groups, eps):  # sum of squares instead of the mean
+        d = x.shape[-1] // groups
+        return good(x, groups, eps) / math.sqrt(d)
+
+    def interleaved(x, groups, eps):  # shards as strided columns
+        x = np.asarray(x, np.float64)
+        out = np.empty_like(x)
+        for g in range(groups):
+            blk = x[..., g::groups]
+            out[..., g::groups] = blk / np.sqrt((blk * blk).mean(axis=-1, keepdims=True) + eps)
+        return out
+
+    for bad in (norm_over_width, no_mean, interleaved):
+        monkeypatch.setattr(O, "rms_norm_groups_ref", bad)
+        got = O.cache_row_ref(a, 4, False, 1e-6)
+        want = _cache_row_bruteforce(a, 4, False, 1e-6)
+        assert np.abs(got - np.asarray(want)).max() > 1e-3, bad.__name__
+    monkeypatch.setattr(O, "rms_norm_groups_ref", good)

@@ -1,0 +1,109 @@
+"""GPU parity of the PCA reparameterisation against the float64 oracle: the
+calibration covariance, the rotation x -> x U of q and cache rows, decode on
+rotated inputs, the G=1 invariance after rotating back, and U folded into
+W_uv.  U is the oracle's basis rounded to bf16; the oracle is given the same
+rounded values, so only accumulation order and the bf16 store differ."""
+
+import numpy as np
+import pytest
+import torch
+
+import mla_latent_kv_dim_b200 as tp
+from mla_latent_kv_dim_b200.workloads import make_inputs
+from oracle import tpla_oracle as O
+from parity import as_f64, assert_lse_close, assert_out_close, oracle_rows, to_device, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def calib():
+    w = make_inputs(4, 16, [4096, 4000, 64, 1000], paged=True, decay=True, seed=31, wuv=True)
+    rows = as_f64(w.cache).reshape(-1, 576)
+    lam, U = O.pca_basis_ref(rows[:, :512])
+    U16 = torch.from_numpy(U).to(torch.bfloat16)
+    return w, rows, U16, as_f64(U16)
+
+
+def test_latent_covariance(cuda_dev, calib):
+    w, rows, _, _ = calib
+    mean, cov = tp.latent_covariance(w.cache.to(cuda_dev))  # [blocks, 64, 576] view
+    torch.cuda.synchronize()
+    m_ref, c_ref = O.latent_covariance_ref(rows[:, :512])
+    got_c, got_m = to_np(cov), to_np(mean)
+    assert np.abs(got_c - c_ref).max() <= 1e-4 * np.abs(c_ref).max()
+    assert np.abs(got_c - c_ref).mean() <= 1e-3 * np.abs(c_ref).mean()
+    assert np.abs(got_m - m_ref).max() <= 1e-4
+
+
+@pytest.mark.parametrize("view,scratch_leads", [("paged", 3), ("flat", 1000), ("flat", 7)])
+def test_rotate_apply(cuda_dev, calib, view, scratch_leads):
+    w, rows, U16, Uq = calib
+    x = w.cache.to(cuda_dev)
+    if view == "flat":
+        x = x.reshape(-1, 576)[:, :]  # [N, 576]
+    per = (x.shape[1] if x.dim() == 3 else 1) * 512
+    scratch = torch.empty(scratch_leads * per, dtype=torch.float32, device=cuda_dev)
+    before = x.clone()
+    tp.rotate_apply(x, U16.to(cuda_dev), scratch=scratch)
+    torch.cuda.synchronize()
+    got = to_np(x).reshape(-1, 576)
+    ref = O.pca_rotate_ref(rows, Uq)
+    ref16 = as_f64(torch.from_numpy(ref).to(torch.bfloat16))
+    assert np.array_equal(got[:, 512:], to_np(before).reshape(-1, 576)[:, 512:])
+    # one bf16 rounding of an f32 sum of 512 exact products: within one bf16
+    # step of the rounded oracle plus the f32 accumulation bound (with slack)
+    terms = np.abs(rows[:, :512]) @ np.abs(Uq)
+    tol = np.abs(ref16[:, :512]) * 2.0 ** -7 + terms * 2.0 ** -13
+    assert np.all(np.abs(got[:, :512] - ref16[:, :512]) <= tol)
+    assert_out_close(got[:, :512], ref16[:, :512])
+
+
+def test_decode_on_pca_rotated_inputs_and_g1_invariance(cuda_dev, calib):
+    w, rows, U16, Uq = calib
+    d = to_device(w, cuda_dev)
+    Ud = U16.to(cuda_dev)
+    tp.rotate_apply(d["q"], Ud)
+    tp.rotate_apply(d["cache"], Ud)
+    torch.cuda.synchronize()
+    qr = to_np(d["q"])
+    cache_r = to_np(d["cache"])
+    rows_r = []
+    for b in range(w.B):
+        L = int(w.seq_lens[b])
+        n = (L + 63) // 64
+        rows_r.append(cache_r[w.page_table[b, :n].long().numpy()].reshape(n * 64, 576)[:L])
+    # TPLA G=2 on the rotated inputs, against the oracle on the same bf16 values
+    out, lse = tp.decode(d["q"], d["cache"], d["seq_lens"], d["page_table"], 2, "replicate",
+                         w.scale)
+    torch.cuda.synchronize()
+    ro, rl = O.tpla_decode_ref(qr, rows_r, 2, "replicate", np.float32(w.scale))
+    assert_out_close(to_np(out), ro)
+    assert_lse_close(to_np(lse), rl)
+    # G=1 on the rotated inputs, rotated back: parity with the oracle doing the same
+    out1, lse1 = tp.decode(d["q"], d["cache"], d["seq_lens"], d["page_table"], 1, "replicate",
+                           w.scale)
+    torch.cuda.synchronize()
+    back = O.pca_unrotate_ref(to_np(out1), Uq)
+    o1, l1 = O.tpla_decode_ref(qr, rows_r, 1, "replicate", np.float32(w.scale))
+    assert_out_close(back, O.pca_unrotate_ref(o1, Uq))
+    assert_lse_close(to_np(lse1), l1)
+    # and it is exact MLA on the original inputs up to U's bf16 rounding: U U^T
+    # differs from I by ~5e-3 (spectral norm) and the rotated rows are rounded
+    # to bf16, which on these inputs puts the oracle itself at 5.2e-3 (max) and
+    # 4.3e-3 (mean) relative error; allowed here: 2e-2 and 1e-2
+    r0, l0 = O.tpla_decode_ref(as_f64(w.q), oracle_rows(w), 1, "replicate", np.float32(w.scale))
+    err = np.abs(back - r0)
+    assert err.max() <= 2e-2 * np.abs(r0).max()
+    assert err.mean() <= 1e-2 * np.abs(r0).mean()
+    # U^T folded into W_uv (rotate the rows of W^T), then y from the rotated output
+    W = w.W_uv.to(cuda_dev)
+    Wt = W.transpose(1, 2).contiguous()
+    tp.rotate_apply(Wt, Ud)
+    Wf = Wt.transpose(1, 2).contiguous()
+    y = tp.vup_combine(out1, Wf)
+    torch.cuda.synchronize()
+    Wf_ref = as_f64(torch.from_numpy(O.fold_vup_ref(as_f64(w.W_uv), Uq)).to(torch.bfloat16))
+    assert_out_close(to_np(Wf), Wf_ref, what="folded W_uv (bf16)")
+    assert_out_close(to_np(y), O.vup_ref(to_np(out1), to_np(Wf)), what="y")
+    assert tp.device_status() == 0
