@@ -285,6 +285,44 @@ TPLA_API int tpla_covariance_finalize(const tpla_tensor* C, const tpla_tensor* s
 TPLA_API int tpla_rotate_apply(tpla_tensor* buf, const tpla_tensor* U, void* scratch,
                                size_t scratch_bytes, tpla_stream_t stream);
 
+/*
+ * tpla_cache_append -- store each request's new token in the latent cache,
+ * normalised the way the shards read it.  The review of arXiv 2508.15881
+ * (key machinery): the stored latent is the RMS-normalised down-projection
+ * (its gain absorbed into the up-projections, like the rotation U), and in
+ * TPLA every rank normalises its own slice, which Condition 1 asks to track
+ * the global norm; its referee report calls Proposition 1 (RMSNorm commutes
+ * with an orthogonal transform) correct.  The feature request ("Directions
+ * under investigation") applies the Hadamard reparameterisation on this
+ * path (kv_a_layernorm).
+ *   kv_new      [B, 576] bf16 or f32, rows 16-byte aligned: columns 0..511
+ *               the token's latent before normalisation, 512..575 its
+ *               position-encoded rope key (stored as given).
+ *   positions   [B] int32: token index each request writes (its length
+ *               before this token, for appending).
+ *   page_table  [B, max_pages] int32 (paged cache) or NULL (contiguous).
+ *   kv_cache    paged [num_blocks, 64, 576] or contiguous [B, Lmax, 576]
+ *               bf16, the layout tpla_decode_ex reads; 16-byte aligned rows.
+ *   norm_groups 1: one RMS over all 512 latent columns (exact MLA); 2, 4 or
+ *               8: each contiguous shard of 512 / norm_groups columns
+ *               divided by its own RMS (one TPLA rank per shard).
+ *   hadamard    1: rotate the latent by the orthonormal Walsh-Hadamard matrix
+ *               (tpla_hadamard_apply's) before the norm; 0: no rotation.
+ *   eps         >= 0, added to each mean square.
+ * Stored row: latent x (rotated if asked), each shard x_g / sqrt(mean(x_g^2)
+ * + eps), f32 arithmetic, rounded once to bf16; rope copied.  A position
+ * outside the cache or a page id outside [0, num_blocks) is not written: the
+ * kernel records TPLA_ERR_DEVICE_BOUNDS (tpla_get_device_status).  Nothing
+ * else of the cache is touched.  Asynchronous on `stream`; allocates nothing.
+ * Errors before any launch: TPLA_ERR_INVALID_ARG (shapes, dtypes, strides,
+ * alignment, norm_groups, hadamard, eps); TPLA_ERR_UNSUPPORTED (B > 2^20,
+ * paged cache with pages other than 64 tokens).
+ */
+TPLA_API int tpla_cache_append(const tpla_tensor* kv_new, const tpla_tensor* positions,
+                               const tpla_tensor* page_table, tpla_tensor* kv_cache,
+                               int norm_groups, int hadamard, float eps,
+                               tpla_stream_t stream);
+
 /* Human-readable name of a tpla_status code (static string). */
 TPLA_API const char* tpla_error_string(int status);
 

@@ -5,11 +5,12 @@ CUDA kernels for sm_100a.  This package holds the ctypes binding
 (``_native``), the in-tree build (``build``) and the seeded synthetic
 workloads (``workloads``).
 """
-from ._native import (TplaError, decode, decode_simple, decode_workspace_size,  # noqa: F401
+from ._native import (TplaError, cache_append, decode, decode_simple,  # noqa: F401
+                      decode_workspace_size,
                       device_status, error_string, hadamard_apply, latent_covariance,
                       launch_count, lse_merge, lib, rotate_apply, selftest_wait_timeout,
                       version, vup_combine)
 
-__all__ = ["TplaError", "decode", "decode_simple", "decode_workspace_size", "device_status",
+__all__ = ["TplaError", "cache_append", "decode", "decode_simple", "decode_workspace_size", "device_status",
            "selftest_wait_timeout", "latent_covariance", "rotate_apply",
            "error_string", "hadamard_apply", "launch_count", "lse_merge", "lib", "version", "vup_combine"]

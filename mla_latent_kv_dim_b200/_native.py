@@ -80,11 +80,13 @@ def lib() -> ctypes.CDLL:
             L.tpla_covariance_finalize.argtypes = [T, T, ctypes.c_int64, T, T, ctypes.c_void_p]
             L.tpla_rotate_apply.argtypes = [T, T, ctypes.c_void_p, ctypes.c_size_t,
                                             ctypes.c_void_p]
+            L.tpla_cache_append.argtypes = [T, T, T, T, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_float, ctypes.c_void_p]
             for f in ("tpla_decode_ex", "tpla_decode", "tpla_decode_workspace_size",
                       "tpla_lse_merge", "tpla_hadamard_apply", "tpla_vup_combine",
                       "tpla_last_cuda_error", "tpla_get_device_status", "tpla_version",
                       "tpla_selftest_wait_timeout", "tpla_latent_covariance",
-                      "tpla_covariance_finalize", "tpla_rotate_apply"):
+                      "tpla_covariance_finalize", "tpla_rotate_apply", "tpla_cache_append"):
                 getattr(L, f).restype = ctypes.c_int
             L.tpla_launch_count.restype = ctypes.c_int64
             _lib = L
@@ -280,6 +282,21 @@ def rotate_apply(buf, U, scratch=None, stream=None):
                                  scratch.numel() * scratch.element_size(), _stream(stream))
     _check("tpla_rotate_apply", rc)
     return buf
+
+
+def cache_append(kv_new, positions, page_table, kv_cache, norm_groups=1, hadamard=False,
+                 eps=1e-6, stream=None):
+    """Store each request's new token row (``kv_new`` [B, 576]: latent before
+    its RMS normalisation, then the rope key) into ``kv_cache`` at token
+    ``positions[b]``, normalised over ``norm_groups`` shards, optionally
+    rotated first (tpla_cache_append).  In place on ``kv_cache``."""
+    _on_current_device(kv_new, positions, page_table, kv_cache)
+    rc = lib().tpla_cache_append(_ref(desc(kv_new)), _ref(desc(positions)),
+                                 _ref(desc(page_table)) if page_table is not None else None,
+                                 _ref(desc(kv_cache)), int(norm_groups), 1 if hadamard else 0,
+                                 ctypes.c_float(eps), _stream(stream))
+    _check("tpla_cache_append", rc)
+    return kv_cache
 
 
 def device_status(stream=None) -> int:

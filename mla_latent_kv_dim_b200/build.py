@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libtpla.so")
 SOURCES = ["api.cu", "decode_generic.cu", "decode_sm100.cu", "merge.cu", "hadamard.cu",
-           "vup.cu", "noalloc.cu", "pca.cu"]
+           "vup.cu", "noalloc.cu", "pca.cu", "append.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -403,6 +403,49 @@ int tpla_rotate_apply(tpla_tensor* buf, const tpla_tensor* U, void* scratch,
   return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
 }
 
+int tpla_cache_append(const tpla_tensor* kv_new, const tpla_tensor* positions,
+                      const tpla_tensor* page_table, tpla_tensor* kv_cache, int norm_groups,
+                      int hadamard, float eps, tpla_stream_t stream) {
+  if (!kv_new || (kv_new->dtype != TPLA_BF16 && kv_new->dtype != TPLA_F32))
+    return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(kv_new, kv_new->dtype, 2) || kv_new->shape[1] != kWidth)
+    return TPLA_ERR_INVALID_ARG;
+  const int64_t B = kv_new->shape[0];
+  const int64_t esz = kv_new->dtype == TPLA_BF16 ? 2 : 4;
+  if (B > 0 && (!aligned16(kv_new->data) || (kv_new->stride[0] * esz) % 16))
+    return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(positions, TPLA_I32, 1) || positions->shape[0] != B)
+    return TPLA_ERR_INVALID_ARG;
+  if (!(norm_groups == 1 || norm_groups == 2 || norm_groups == 4 || norm_groups == 8))
+    return TPLA_ERR_INVALID_ARG;
+  if (!(hadamard == 0 || hadamard == 1) || !isfinite(eps) || eps < 0.f)
+    return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(kv_cache, TPLA_BF16, 3) || kv_cache->shape[2] != kWidth)
+    return TPLA_ERR_INVALID_ARG;
+  if (!aligned16(kv_cache->data) || kv_cache->stride[0] % 8 || kv_cache->stride[1] % 8)
+    return TPLA_ERR_INVALID_ARG;
+  int max_pages = 0;
+  if (page_table) {
+    if (!check_tensor(page_table, TPLA_I32, 2) || page_table->shape[0] != B)
+      return TPLA_ERR_INVALID_ARG;
+    if (kv_cache->shape[1] != kBlock) return TPLA_ERR_UNSUPPORTED;
+    if (page_table->shape[1] > (1 << 24)) return TPLA_ERR_UNSUPPORTED;
+    max_pages = (int)page_table->shape[1];
+  } else if (kv_cache->shape[0] != B) {
+    return TPLA_ERR_INVALID_ARG;
+  }
+  if (B > (1 << 20)) return TPLA_ERR_UNSUPPORTED;
+  if (B == 0) return TPLA_OK;
+  cudaError_t e = launch_cache_append(
+      kv_new->data, kv_new->dtype == TPLA_BF16, kv_new->stride[0],
+      reinterpret_cast<const int*>(positions->data),
+      page_table ? reinterpret_cast<const int*>(page_table->data) : nullptr,
+      page_table ? page_table->stride[0] : 0, max_pages, kv_cache->shape[0], kv_cache->shape[1],
+      kv_cache->data, kv_cache->stride[0], kv_cache->stride[1], (int)B, norm_groups, hadamard,
+      eps, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
+}
+
 const char* tpla_error_string(int status) {
   switch (status) {
     case TPLA_OK: return "ok";
@@ -427,10 +470,12 @@ int tpla_get_device_status(tpla_stream_t stream, int* status) {
   if (e != cudaSuccess) return cuda_fail(e);
   e = status_read_clear_sm100(&b);
   if (e != cudaSuccess) return cuda_fail(e);
-  int c = 0;
+  int c = 0, d = 0;
   e = status_read_clear_vup(&c);
   if (e != cudaSuccess) return cuda_fail(e);
-  *status = a != 0 ? a : (b != 0 ? b : c);
+  e = status_read_clear_append(&d);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *status = a != 0 ? a : (b != 0 ? b : (c != 0 ? c : d));
   return TPLA_OK;
 }
 

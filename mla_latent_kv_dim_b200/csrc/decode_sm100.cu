@@ -133,6 +133,8 @@ struct Params {
   float* part_o;  // [slots, H, W]
   float* part_l;  // [slots, H, nsh]
   int W;
+  int tile_tok;  // tokens per schedule tile: 256 (pair kernel) or 128 (shard kernel)
+  int ring;      // shard kernel: ring slots
   int mode;  // 0 = balanced persistent ranges, 1 = explicit equal splits
   int P;     // clusters
   int S;     // explicit splits
@@ -150,7 +152,7 @@ __device__ __forceinline__ int req_len(const Params& p, int b) {
 }
 
 __device__ __forceinline__ int req_tiles(const Params& p, int b) {
-  return (req_len(p, b) + kTileTok - 1) / kTileTok;
+  return (req_len(p, b) + p.tile_tok - 1) / p.tile_tok;
 }
 
 struct Segment {
@@ -923,6 +925,466 @@ tpla_decode_sm100_kernel(const __grid_constant__ CUtensorMap qmap,
   }
 }
 
+// ================================================================ shard kernel (G >= 2)
+//
+// One CTA computes one TPLA shard, as one tensor-parallel rank would: all
+// 128 heads of the request in one single-CTA MMA (M = 128), over the shard's
+// latent columns and its rope columns.  The CTAs of a token range (one per
+// shard) are launched next to each other and run together, so the rope chunk
+// they share is read from DRAM once and from L2 by the others.  Unlike the
+// pair kernel, every cache byte is staged into shared memory once: the tile's
+// latent chunks stay in the ring from QK^T through P.V (the P.V operand is
+// MN-major over the same bytes), and P lives in tensor memory over the S it
+// came from, so the ring gets the shared memory the pair kernel spends on P
+// and on re-reading the peer's tokens.
+//  * Tiles of 128 tokens (two pages).  A stage is chunk c of both pages:
+//    [64 rows][64 bf16] x 2, 16 KB, in the 128-byte swizzle.  Per tile the
+//    rope chunk first (its slot is free again as soon as QK^T has read it),
+//    then the shard's d/64 latent chunks.  With 9 slots at G = 2 (5 stages
+//    per tile) the loads of tile i then wait only for P.V of tile i - 2 and
+//    QK^T of tile i - 1: two tiles in flight.
+//  * QK^T: M = 128 heads, N = 128 tokens, K-steps over the stage; S in TMEM
+//    (two buffers of 128 columns).  P.V: M = 128, N = 64 latent columns per
+//    chunk, K = 128 tokens, A = P read from TMEM; O (d <= 256 columns) in
+//    TMEM.  The rope slot is released after QK^T, latent slots after P.V.
+//  * Warps: 0 QK^T issuer (and TMEM allocation), 1 P.V issuer, 2-3 TMA
+//    producers, 4-7 softmax: one thread per head (its TMEM lane) over all
+//    128 tokens of a tile, so the row max needs no exchange between threads
+//    and P overwrites only the thread's own lane of S.
+namespace shd {
+
+constexpr int kTile = 128;
+constexpr int kStage = 16384;
+constexpr int kQChunkBytes = 16384;  // [128 heads][64 columns] bf16
+constexpr int kMaxRing = 12;
+constexpr int kWarpQK = 0, kWarpPV = 1, kWarpProd0 = 2, kWarpSm0 = 4;  // producers: warps 2, 3
+constexpr int kSoftmaxWarps = 4;
+constexpr int kThreads = 32 * (kWarpSm0 + kSoftmaxWarps);
+constexpr uint32_t kColS = 0;    // S / P buffers: [0, 128), [128, 256)
+constexpr uint32_t kColO = 256;  // O: d <= 256 columns
+constexpr int kNumBars = 2 * kMaxRing + 8;
+constexpr int kMiscBytes = kNumBars * 8 + 16;
+constexpr int kSmemBytes = 232448;  // the per-block maximum; the ring takes what Q leaves
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 64, false, true);
+
+struct Bars {
+  uint32_t base;
+  __device__ uint32_t full(int s) const { return base + 8 * s; }
+  __device__ uint32_t empty(int s) const { return base + 8 * (kMaxRing + s); }
+  __device__ uint32_t q_full() const { return base + 8 * (2 * kMaxRing); }
+  __device__ uint32_t q_empty() const { return base + 8 * (2 * kMaxRing + 1); }
+  __device__ uint32_t s_full(int i) const { return base + 8 * (2 * kMaxRing + 2 + i); }
+  __device__ uint32_t p_full(int i) const { return base + 8 * (2 * kMaxRing + 4 + i); }
+  __device__ uint32_t pv_done(int i) const { return base + 8 * (2 * kMaxRing + 6 + i); }
+};
+
+struct Layout {  // shared-memory offsets (bytes from the 1 KB aligned base)
+  uint32_t ring, bars, tmem_slot, abort;
+};
+
+// q chunks (rope first, then the shard's latent chunks), ring, barriers
+__device__ __forceinline__ Layout layout(const Params& p) {
+  Layout L;
+  L.ring = (uint32_t)(p.dq + 1) * kQChunkBytes;
+  L.bars = L.ring + (uint32_t)p.ring * kStage;
+  L.tmem_slot = L.bars + kNumBars * 8;
+  L.abort = L.tmem_slot + 4;
+  return L;
+}
+
+// cache / q chunk of stage `st` of a tile: the rope chunk, then the latent
+__device__ __forceinline__ int stage_chunk(const Params& p, int g, int st) {
+  return st == 0 ? kRopeChunk : g * p.dq + st - 1;
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+      :
+      : "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2),
+        "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];"
+      :
+      : "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem] B[smem]^T (single CTA), descriptors as 32-bit halves
+__device__ __forceinline__ void mma_ss(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                       uint32_t b_hi, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}"
+      :
+      : "r"(d), "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] B[smem]^T: A (M x 16) in TMEM, lane = row, 16-bit
+// elements packed two per 32-bit column.
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                       uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}"
+      :
+      : "r"(d), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// CTA `cta` of the grid: token range `range`, shard index `i` among the
+// range's nsh shards.
+__device__ __forceinline__ void cta_role(const Params& p, int cta, int& range, int& i) {
+  range = cta / p.nsh;
+  i = cta % p.nsh;
+}
+
+__device__ void producer(const Params& p, const CUtensorMap* qmap, const CUtensorMap* kvmap,
+                         int range, int g, int pid, uint32_t sbase, const Layout& L,
+                         const Bars& bars, volatile int* abort_flag) {
+  const int lane = threadIdx.x & 31;
+  Cursor cur;
+  seg_begin(p, range, cur);
+  Segment s;
+  PageWindow win;
+  uint32_t n = 0, qloads = 0;
+  const int nq = p.dq + 1;
+  while (seg_next(p, range, cur, s)) {
+    const int ntiles = s.t_hi - s.t_lo;
+    if (ntiles == 0) continue;
+    if (pid == 0) {  // the shard's q, once the previous segment's QK^T is done
+      if (qloads > 0 && !wait_bar_warp(bars.q_empty(), (qloads - 1) & 1, abort_flag)) return;
+      if (lane == 0) mbar_arrive_expect_tx(bars.q_full(), nq * kQChunkBytes);
+      __syncwarp();
+      if (lane < nq)
+        tma_load_3d(sbase + lane * kQChunkBytes, qmap, 64 * stage_chunk(p, g, lane), 0, s.b,
+                    bars.q_full());
+    }
+    ++qloads;
+    for (int j = 0; j < ntiles; ++j) {
+      const int t = s.t_lo + j;
+      int blk0 = 0, blk1 = 0;
+      if (p.paged) {
+        blk0 = win.get(p, s, 2 * t, lane);
+        blk1 = win.get(p, s, 2 * t + 1, lane);
+      }
+      for (int st = 0; st < nq; ++st) {
+        const uint32_t me = n++;
+        const uint32_t slot = me % (uint32_t)p.ring;
+        if ((slot & 1u) != (uint32_t)pid) continue;
+        if (me >= (uint32_t)p.ring &&
+            !wait_bar_warp(bars.empty(slot), ((me / p.ring) - 1) & 1, abort_flag))
+          return;
+        if (lane == 0) mbar_arrive_expect_tx(bars.full(slot), kStage);
+        __syncwarp();
+        if (lane < 2) {  // one page per lane
+          const int c = stage_chunk(p, g, st);
+          const uint32_t dst = sbase + L.ring + slot * kStage + lane * (kStage / 2);
+          if (p.paged)
+            tma_load_4d(dst, kvmap, 0, 0, c, lane == 0 ? blk0 : blk1, bars.full(slot));
+          else
+            tma_load_4d(dst, kvmap, 0, kTile * t + 64 * lane, c, s.b, bars.full(slot));
+        }
+      }
+    }
+  }
+}
+
+__device__ void qk_issuer(const Params& p, int range, int g, uint32_t sbase, uint32_t tmem,
+                          const Layout& L, const Bars& bars, volatile int* abort_flag) {
+  Cursor cur;
+  seg_begin(p, range, cur);
+  Segment s;
+  uint32_t n = 0, qloads = 0, U = 0, parity = 0;
+  const int nq = p.dq + 1;
+  int rk0, rk1;
+  rope_steps(p, g, rk0, rk1);
+  const uint64_t dQ = sw128_desc(sbase, 16, 1024);
+  const uint64_t dR = sw128_desc(sbase + L.ring, 16, 1024);
+  const uint32_t q_lo = (uint32_t)dQ, q_hi = (uint32_t)(dQ >> 32);
+  const uint32_t r_lo = (uint32_t)dR, r_hi = (uint32_t)(dR >> 32);
+  constexpr uint32_t kQDesc = kQChunkBytes >> 4, kStageDesc = kStage >> 4;
+  while (seg_next(p, range, cur, s)) {
+    const int ntiles = s.t_hi - s.t_lo;
+    if (ntiles == 0) continue;
+    if (!wait_bar(bars.q_full(), qloads & 1, abort_flag)) return;
+    ++qloads;
+    tc_fence_after();
+    for (int j = 0; j < ntiles; ++j, ++U) {
+      // S[U & 1] (with the P over it) is free once P.V of tile U - 2 completed
+      if (U >= 2 && !wait_bar(bars.pv_done(U & 1), ((U - 2) >> 1) & 1, abort_flag)) return;
+      tc_fence_after();
+      const uint32_t dS = tmem + kColS + 128 * (U & 1);
+      uint32_t acc = 0;
+      for (int st = 0; st < nq; ++st) {
+        const uint32_t slot = (n + st) % (uint32_t)p.ring;
+        if (!wait_bar(bars.full(slot), (parity >> slot) & 1u, abort_flag)) return;
+        parity ^= 1u << slot;
+        const uint32_t a = q_lo + (uint32_t)st * kQDesc;
+        const uint32_t b = r_lo + slot * kStageDesc;
+        if (st > 0) {
+          mma_ss(dS, a, q_hi, b, r_hi, kIdescQK, acc);
+          mma_ss(dS, a + 2, q_hi, b + 2, r_hi, kIdescQK, 1u);
+          mma_ss(dS, a + 4, q_hi, b + 4, r_hi, kIdescQK, 1u);
+          mma_ss(dS, a + 6, q_hi, b + 6, r_hi, kIdescQK, 1u);
+          acc = 1;
+        } else {
+          for (int kk = rk0; kk < rk1; ++kk) {
+            mma_ss(dS, a + 2 * kk, q_hi, b + 2 * kk, r_hi, kIdescQK, acc);
+            acc = 1;
+          }
+          commit(bars.empty(slot));  // the rope chunk is needed by QK^T only
+        }
+      }
+      commit(bars.s_full(U & 1));
+      n += nq;
+    }
+    commit(bars.q_empty());
+  }
+}
+
+__device__ void pv_issuer(const Params& p, int range, uint32_t sbase, uint32_t tmem,
+                          const Layout& L, const Bars& bars, volatile int* abort_flag) {
+  Cursor cur;
+  seg_begin(p, range, cur);
+  Segment s;
+  uint32_t n = 0, U = 0;
+  const int nq = p.dq + 1;
+  // MN-major V operand: rows = tokens (K), 64 latent columns per 128-byte row
+  const uint64_t dV = sw128_desc(sbase + L.ring, kStage / 2, 1024);
+  const uint32_t v_lo = (uint32_t)dV, v_hi = (uint32_t)(dV >> 32);
+  constexpr uint32_t kStageDesc = kStage >> 4;
+  while (seg_next(p, range, cur, s)) {
+    const int ntiles = s.t_hi - s.t_lo;
+    if (ntiles == 0) continue;
+    for (int j = 0; j < ntiles; ++j, ++U) {
+      if (!wait_bar(bars.p_full(U & 1), (U >> 1) & 1, abort_flag)) return;
+      tc_fence_after();
+      const uint32_t pa = tmem + kColS + 128 * (U & 1);  // P: 64 columns of bf16 pairs
+      for (int c = 0; c < p.dq; ++c) {
+        const uint32_t slot = (n + 1 + c) % (uint32_t)p.ring;
+        const uint32_t b = v_lo + slot * kStageDesc;
+        const uint32_t dO = tmem + kColO + 64 * c;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // 16 tokens per step: P +8 columns, V +2 KB
+          mma_ts(dO, pa + 8 * k, b + 128 * k, v_hi, kIdescPV, (j | k) != 0);
+        commit(bars.empty(slot));
+      }
+      commit(bars.pv_done(U & 1));
+      n += nq;
+    }
+  }
+}
+
+__device__ void softmax(const Params& p, int range, int i_sh, int g, uint32_t tmem,
+                        const Bars& bars, volatile int* abort_flag) {
+  const int w = (int)(threadIdx.x >> 5);
+  const int head = 32 * (w & 3) + (int)(threadIdx.x & 31);  // = this thread's TMEM lane
+  const uint32_t lane_base = (uint32_t)(32 * (w & 3)) << 16;
+  const int col_base = p.shard < 0 ? g * p.d : 0;
+  Cursor cur;
+  seg_begin(p, range, cur);
+  Segment s;
+  uint32_t U = 0;
+  while (seg_next(p, range, cur, s)) {
+    const int ntiles = s.t_hi - s.t_lo;
+    if (ntiles == 0) {  // empty chunk: out 0, lse -inf
+      float z[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) z[j] = 0.f;
+      for (int c0 = 0; c0 < p.d; c0 += 32) write_out_row(p, s, head, col_base + c0, z, 0.f);
+      write_lse(p, s, head, i_sh, -INFINITY);
+      continue;
+    }
+    float m = -INFINITY, l = 0.f;
+    for (int j = 0; j < ntiles; ++j, ++U) {
+      const int t = s.t_lo + j;
+      if (!wait_bar(bars.s_full(U & 1), (U >> 1) & 1, abort_flag)) return;
+      tc_fence_after();
+      const uint32_t sb = tmem + lane_base + kColS + 128 * (U & 1);
+      float x[128];
+      {
+        uint32_t r[4][32];
+        tmem_ld32(sb, r[0]);
+        tmem_ld32(sb + 32, r[1]);
+        tmem_ld32(sb + 64, r[2]);
+        tmem_ld32(sb + 96, r[3]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 128; ++k) x[k] = __uint_as_float(r[k >> 5][k & 31]);
+      }
+      if (p.negate) {
+#pragma unroll
+        for (int k = 0; k < 128; ++k) x[k] = -x[k];
+      }
+      const int nv = max(0, min(kTile, s.L - kTile * t));
+      if (nv < kTile) {  // warp-uniform: the request's last tile
+#pragma unroll
+        for (int k = 0; k < 128; ++k) x[k] = k < nv ? x[k] : -INFINITY;
+      }
+      float mx0 = fmaxf(x[0], x[1]), mx1 = fmaxf(x[2], x[3]);
+#pragma unroll
+      for (int k = 4; k < 128; k += 4) {
+        mx0 = fmaxf(mx0, fmaxf(x[k], x[k + 1]));
+        mx1 = fmaxf(mx1, fmaxf(x[k + 2], x[k + 3]));
+      }
+      const float mx = fmaxf(mx0, mx1) * p.scale_log2;
+      float factor = 1.f;
+      int resc = 0;
+      if (m == -INFINITY) {
+        m = mx;
+      } else if (mx > m + kRescaleThreshold) {
+        factor = ex2(m - mx);
+        m = mx;
+        resc = 1;
+      }
+      l *= factor;
+      if (__any_sync(0xffffffffu, resc)) {
+        // O was last written by P.V of tile U - 1 (not the first of the segment)
+        if (!wait_bar(bars.pv_done((U - 1) & 1), ((U - 1) >> 1) & 1, abort_flag)) return;
+        tc_fence_after();
+        for (int c0 = 0; c0 < p.d; c0 += 32) {
+          const uint32_t ta = tmem + lane_base + kColO + c0;
+          uint32_t o[32];
+          tmem_ld32(ta, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * factor);
+          tmem_st32(ta, o);
+        }
+        tmem_wait_st();
+      }
+      // P = 2^(x - m) in bf16 (masked tokens give 0); l sums the rounded values.
+      // P goes over this lane's own S columns [0, 64): the thread has read them.
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-m, -m);
+      uint64_t ls2 = f2_pack(0.f, 0.f);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          float e0, e1;
+          f2_unpack(f2_fma(f2_pack(x[64 * h + 2 * k], x[64 * h + 2 * k + 1]), sc2, nm2), e0, e1);
+          const uint32_t u = cvt_bf16x2(ex2(e0), ex2(e1));
+          ls2 = f2_add(ls2, f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u)));
+          pk[k] = u;
+        }
+        tmem_st32(sb + 32 * h, pk);
+      }
+      float ls0, ls1;
+      f2_unpack(ls2, ls0, ls1);
+      l += ls0 + ls1;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) arrive(bars.p_full(U & 1));
+    }
+    // epilogue: the segment's last P.V done
+    if (!wait_bar(bars.pv_done((U - 1) & 1), ((U - 1) >> 1) & 1, abort_flag)) return;
+    tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const float lse = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+    for (int c0 = 0; c0 < p.d; c0 += 32) {
+      uint32_t o[32];
+      tmem_ld32(tmem + lane_base + kColO + c0, o);
+      tmem_wait_ld();
+      write_out_row(p, s, head, col_base + c0, reinterpret_cast<const float*>(o), inv);
+    }
+    write_lse(p, s, head, i_sh, lse);
+    tc_fence_before();
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+tpla_decode_shard_kernel(const __grid_constant__ CUtensorMap qmap,
+                         const __grid_constant__ CUtensorMap kvmap, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Layout L = layout(p);
+  const Bars bars{sbase + L.bars};
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.abort);
+  int range, i_sh;
+  cta_role(p, (int)blockIdx.x, range, i_sh);
+  const int g = shard_of(p, i_sh);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.ring; ++s) {
+      mbar_init(bars.full(s), 1);
+      mbar_init(bars.empty(s), 1);
+    }
+    mbar_init(bars.q_full(), 1);
+    mbar_init(bars.q_empty(), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars.s_full(i), 1);
+      mbar_init(bars.p_full(i), kSoftmaxWarps);
+      mbar_init(bars.pv_done(i), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpProd0 && lane == 0) {
+    tma_prefetch(&qmap);
+    tma_prefetch(&kvmap);
+  }
+  if (warp == kWarpQK) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     sbase + L.tmem_slot)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L.tmem_slot);
+
+  if (warp == kWarpQK) {
+    if (lane == 0) qk_issuer(p, range, g, sbase, tmem, L, bars, abort_flag);
+  } else if (warp == kWarpPV) {
+    if (lane == 0) pv_issuer(p, range, sbase, tmem, L, bars, abort_flag);
+  } else if (warp < kWarpSm0) {
+    producer(p, &qmap, &kvmap, range, g, warp - kWarpProd0, sbase, L, bars, abort_flag);
+  } else {
+    softmax(p, range, i_sh, g, tmem, bars, abort_flag);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpQK) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+}  // namespace shd
+
 // ---------------------------------------------------------------- merge of partial slots
 //
 // Requests cut by a range boundary (or explicitly split) left normalised
@@ -1110,7 +1572,8 @@ __global__ void wait_timeout_selftest_kernel(long long limit) {
 struct DeviceInfo {
   bool init = false;
   bool sm100 = false;
-  int max_clusters = 0;
+  int max_clusters = 0;  // pair kernel: co-resident clusters of 2
+  int shard_ctas = 0;    // shard kernel: co-resident CTAs (one per SM)
 };
 std::mutex g_mu;
 DeviceInfo g_dev[64];
@@ -1180,15 +1643,30 @@ const DeviceInfo& device_info(int dev) {
     return d;
   }
   d.max_clusters = n;
+  if (cudaFuncSetAttribute(shd::tpla_decode_shard_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           shd::kSmemBytes) != cudaSuccess) {
+    cudaGetLastError();
+    return d;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, shd::tpla_decode_shard_kernel,
+                                                    shd::kThreads, shd::kSmemBytes) !=
+          cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
+    return d;
+  }
+  d.shard_ctas = sms * per_sm;
   d.sm100 = true;
   return d;
 }
 
 bool encode_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                uint64_t stride1_bytes, uint64_t stride2_bytes) {
+                uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box_rows = 64) {
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1219,6 +1697,14 @@ int num_slots(const DecodeProblem& p, int num_splits, int max_clusters) {
   return 2 * p.B * num_splits;
 }
 
+// TPLA shards (G >= 2) run on the shard kernel, exact MLA on the pair kernel.
+bool use_shard_kernel(const DecodeProblem& p) { return p.G >= 2; }
+
+// Token ranges of the persistent schedule.
+int num_ranges(const DecodeProblem& p, const DeviceInfo& d) {
+  return use_shard_kernel(p) ? d.shard_ctas / p.n_shards : d.max_clusters;
+}
+
 }  // namespace
 
 void* tensor_map_encoder() {
@@ -1247,7 +1733,7 @@ bool sm100_supported(const DecodeProblem& p, int device) {
 
 size_t sm100_workspace_bytes(const DecodeProblem& p, int num_splits, int device) {
   const DeviceInfo& d = device_info(device);
-  const int slots = num_slots(p, num_splits, d.max_clusters);
+  const int slots = num_slots(p, num_splits, num_ranges(p, d));
   if (slots == 0) return 0;
   const size_t Hg = p.H < 128 ? p.H : 128;  // heads of one launch (128-head groups)
   const size_t o = (size_t)slots * Hg * p.out_width * sizeof(float);
@@ -1255,6 +1741,8 @@ size_t sm100_workspace_bytes(const DecodeProblem& p, int num_splits, int device)
 }
 
 cudaError_t launch_decode_sm100_group(const DecodeProblem& dp, int num_splits, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream);
+cudaError_t launch_decode_shard_group(const DecodeProblem& dp, int num_splits, void* ws,
                                       size_t ws_bytes, cudaStream_t stream);
 
 // More than 128 heads: one launch (plus merge) per group of up to 128 heads,
@@ -1267,10 +1755,78 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
     g.q = reinterpret_cast<const __nv_bfloat16*>(dp.q) + (int64_t)h0 * dp.q_sh;
     g.out = reinterpret_cast<char*>(dp.out) + (int64_t)h0 * dp.o_sh * (dp.out_bf16 ? 2 : 4);
     g.lse = dp.lse ? dp.lse + (int64_t)h0 * dp.l_sh : nullptr;
-    cudaError_t e = launch_decode_sm100_group(g, num_splits, ws, ws_bytes, stream);
+    cudaError_t e = use_shard_kernel(g) ? launch_decode_shard_group(g, num_splits, ws, ws_bytes, stream)
+                                        : launch_decode_sm100_group(g, num_splits, ws, ws_bytes, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+// Fields both kernels share; the caller sets the schedule and the ring.
+void fill_params(const DecodeProblem& dp, Params& p) {
+  p = Params{};
+  p.seq_lens = dp.seq_lens;
+  p.page_table = dp.page_table;
+  p.pt_sb = dp.pt_sb;
+  p.num_blocks = (int)dp.num_blocks;
+  p.cap_tokens = (int)dp.cache_rows;
+  p.paged = dp.page_table != nullptr;
+  p.B = dp.B;
+  p.H = dp.H;
+  p.G = dp.G;
+  p.split_rope = dp.rope_mode == TPLA_ROPE_SPLIT;
+  p.shard = dp.shard;
+  p.nsh = dp.n_shards;
+  p.d = kLatent / dp.G;
+  p.dq = p.d / 64;
+  p.NB = p.d < 256 ? p.d : 256;
+  p.nblk = p.d / p.NB;
+  // The kernels take the row max of the sign-corrected raw scores and apply
+  // |scale| inside exp2.  A zero scale becomes 1e-30 (log2 units): every
+  // finite score then gives exp2(~0) = 1 exactly in f32, as scale 0 does,
+  // while masked (-inf) scores still give 0.
+  p.scale_log2 = fmaxf((float)(fabs((double)dp.scale) * 1.4426950408889634), 1e-30f);
+  p.negate = dp.scale < 0.f;
+  p.out = dp.out;
+  p.out_bf16 = dp.out_bf16;
+  p.o_sb = dp.o_sb;
+  p.o_sh = dp.o_sh;
+  p.lse = dp.lse;
+  p.l_sb = dp.l_sb;
+  p.l_sh = dp.l_sh;
+  p.W = dp.out_width;
+}
+
+// Split slots in the workspace and the schedule (balanced ranges or explicit
+// splits); returns false when the workspace is missing or short.
+bool set_schedule(const DecodeProblem& dp, int num_splits, int ranges, void* ws, size_t ws_bytes,
+                  Params& p) {
+  const int slots = num_slots(dp, num_splits, ranges);
+  if (slots > 0) {
+    const size_t o = (size_t)slots * dp.H * dp.out_width * sizeof(float);
+    const size_t need = ((o + 255) / 256) * 256 + (size_t)slots * dp.H * dp.n_shards * sizeof(float);
+    if (!ws || ws_bytes < need) return false;
+    p.part_o = reinterpret_cast<float*>(ws);
+    p.part_l = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + ((o + 255) / 256) * 256);
+  }
+  if (num_splits == 0) {
+    p.mode = 0;
+    p.P = ranges;
+    p.S = 1;
+  } else {
+    p.mode = 1;
+    p.S = num_splits;
+    p.P = dp.B * num_splits;
+  }
+  return true;
+}
+
+cudaError_t launch_merge(const DecodeProblem& dp, const Params& p, cudaStream_t stream) {
+  if (p.mode == 1 && p.S == 1) return cudaSuccess;
+  sm100_merge_kernel<<<dim3(dp.B, (dp.H + kMergeHeads - 1) / kMergeHeads), kMergeThreads, 0,
+                       stream>>>(p);
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode_sm100_group(const DecodeProblem& dp, int num_splits, void* ws,
@@ -1290,75 +1846,55 @@ cudaError_t launch_decode_sm100_group(const DecodeProblem& dp, int num_splits, v
                                         dp.c_s0 * 2, k);
     if (!ok) return cudaErrorInvalidValue;
   }
-  Params p{};
-  p.seq_lens = dp.seq_lens;
-  p.page_table = dp.page_table;
-  p.pt_sb = dp.pt_sb;
-  p.num_blocks = (int)dp.num_blocks;
-  p.cap_tokens = (int)dp.cache_rows;
-  p.paged = dp.page_table != nullptr;
-  p.B = dp.B;
-  p.H = dp.H;
-  p.G = dp.G;
-  p.split_rope = dp.rope_mode == TPLA_ROPE_SPLIT;
-  p.shard = dp.shard;
-  p.nsh = dp.n_shards;
-  p.d = kLatent / dp.G;
-  p.dq = p.d / 64;
-  p.NB = p.d < 256 ? p.d : 256;
-  p.nblk = p.d / p.NB;
+  Params p;
+  fill_params(dp, p);
   // QK^T stages wait ~2 us to land and then only for the tensor core, so
-  // they get most of the ring; PV stages are consumed at the softmax's pace
-  // measured: G=1 (eight PV stages per tile) wants the deeper PV ring
-  p.qk_slots = dp.G == 1 ? 3 : 4;
+  // they get most of the ring; PV stages are consumed at the softmax's pace.
+  // Measured (slot sweep on the DeepSeek-V3 workload): G=1 (eight PV stages
+  // per tile) and G=4 (two) want 3 QK^T slots, G=2 wants 4.
+  p.qk_slots = dp.G == 2 ? 4 : 3;
   p.pv_slots = kRingSlots - p.qk_slots;
-  // The kernel takes the row max of the sign-corrected raw scores and applies
-  // |scale| inside exp2.  A zero scale becomes 1e-30 (log2 units): every
-  // finite score then gives exp2(~0) = 1 exactly in f32, as scale 0 does,
-  // while masked (-inf) scores still give 0.
-  p.scale_log2 = fmaxf((float)(fabs((double)dp.scale) * 1.4426950408889634), 1e-30f);
-  p.negate = dp.scale < 0.f;
-  p.out = dp.out;
-  p.out_bf16 = dp.out_bf16;
-  p.o_sb = dp.o_sb;
-  p.o_sh = dp.o_sh;
-  p.lse = dp.lse;
-  p.l_sb = dp.l_sb;
-  p.l_sh = dp.l_sh;
-  p.W = dp.out_width;
-  const int slots = num_slots(dp, num_splits, d.max_clusters);
-  if (slots > 0) {
-    const size_t o = (size_t)slots * dp.H * dp.out_width * sizeof(float);
-    const size_t need = ((o + 255) / 256) * 256 + (size_t)slots * dp.H * dp.n_shards * sizeof(float);
-    if (!ws || ws_bytes < need) return cudaErrorInvalidValue;
-    p.part_o = reinterpret_cast<float*>(ws);
-    p.part_l = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + ((o + 255) / 256) * 256);
-  }
-  int clusters;
-  if (num_splits == 0) {
-    p.mode = 0;
-    p.P = d.max_clusters;
-    p.S = 1;
-    clusters = d.max_clusters;
-  } else {
-    p.mode = 1;
-    p.S = num_splits;
-    p.P = dp.B * num_splits;
-    clusters = p.P;
-  }
+  p.tile_tok = kTileTok;
+  if (!set_schedule(dp, num_splits, d.max_clusters, ws, ws_bytes, p)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  launch_config(cfg, attr, clusters, stream);
+  launch_config(cfg, attr, p.P, stream);
   cudaError_t e = cudaLaunchKernelEx(&cfg, tpla_decode_sm100_kernel, qmap, kv[0], kv[1], p);
   count_launch();
   if (e != cudaSuccess) return e;
-  if (p.mode == 0 || p.S > 1) {
-    sm100_merge_kernel<<<dim3(dp.B, (dp.H + kMergeHeads - 1) / kMergeHeads), kMergeThreads, 0,
-                         stream>>>(p);
-    count_launch();
-    e = cudaGetLastError();
-  }
-  return e;
+  return launch_merge(dp, p, stream);
+}
+
+cudaError_t launch_decode_shard_group(const DecodeProblem& dp, int num_splits, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const DeviceInfo& d = device_info(dev);
+  if (!d.sm100 || d.shard_ctas < dp.n_shards) return cudaErrorNotSupported;
+  CUtensorMap qmap, kv;
+  if (!encode_map(&qmap, dp.q, kWidth, dp.H, dp.B, dp.q_sh * 2, dp.q_sb * 2, 128))
+    return cudaErrorInvalidValue;
+  const bool ok = dp.page_table ? encode_kv_map(&kv, dp.cache, kBlock, dp.num_blocks, dp.c_s1 * 2,
+                                                dp.c_s0 * 2, 1)
+                                : encode_kv_map(&kv, dp.cache, dp.cache_rows, dp.B, dp.c_s1 * 2,
+                                                dp.c_s0 * 2, 1);
+  if (!ok) return cudaErrorInvalidValue;
+  Params p;
+  fill_params(dp, p);
+  p.tile_tok = shd::kTile;
+  // the ring takes the shared memory the shard's q leaves
+  const int q_bytes = (p.dq + 1) * shd::kQChunkBytes;
+  int ring = (shd::kSmemBytes - 1024 - q_bytes - shd::kMiscBytes) / shd::kStage;
+  p.ring = ring > shd::kMaxRing ? shd::kMaxRing : ring;
+  if (p.ring < 2) return cudaErrorNotSupported;
+  if (!set_schedule(dp, num_splits, num_ranges(dp, d), ws, ws_bytes, p))
+    return cudaErrorInvalidValue;
+  const int ctas = p.P * p.nsh;
+  shd::tpla_decode_shard_kernel<<<ctas, shd::kThreads, shd::kSmemBytes, stream>>>(qmap, kv, p);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_merge(dp, p, stream);
 }
 
 cudaError_t launch_wait_timeout_selftest(long long cycles, cudaStream_t stream) {

@@ -93,6 +93,13 @@ cudaError_t launch_covariance_finalize(const float* C, int64_t c_s0, const float
 cudaError_t launch_rotate(void* x, int64_t B, int64_t H, int64_t sb, int64_t sh, const void* U,
                           float* scratch, int64_t chunk_b, cudaStream_t stream);
 
+// ---------------------------------------------------------------- cache append
+cudaError_t launch_cache_append(const void* kv_new, int in_bf16, int64_t n_sb, const int* positions,
+                                const int* page_table, int64_t pt_sb, int max_pages,
+                                int64_t num_blocks, int64_t cap_rows, void* cache, int64_t c_s0,
+                                int64_t c_s1, int B, int groups, int hadamard, float eps,
+                                cudaStream_t stream);
+
 // ---------------------------------------------------------------- launch counter
 // Called once per kernel launch by every launcher.
 void count_launch(int n = 1);
@@ -103,6 +110,7 @@ void count_launch(int n = 1);
 cudaError_t status_read_clear_generic(int* code);
 cudaError_t status_read_clear_sm100(int* code);
 cudaError_t status_read_clear_vup(int* code);
+cudaError_t status_read_clear_append(int* code);
 cudaError_t launch_wait_timeout_selftest(long long cycles, cudaStream_t stream);
 
 }  // namespace tpla

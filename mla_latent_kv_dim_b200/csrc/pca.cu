@@ -17,11 +17,11 @@
 //    per output at the end of a CTA's row chunk.  Calibration sets are small
 //    (tens of thousands of rows), so plain FMA is enough.
 //  * covariance_finalize_kernel: mean = s / n, cov = C / n - mean mean^T.
-//  * rotation: the V-up GEMM (same contraction, U shared by every row through
-//    a zero head stride) writes x U in f32 to caller scratch; a store kernel
-//    rounds it to bf16 back into the rows.  The GEMM reads every source row
-//    before the store of the same chunk starts (stream order), so the
-//    rotation is in place.
+//  * rotation: the V-up kernel (the same contraction: the rows play the
+//    requests of one head, U's two 256-column halves the V dimension) writes
+//    x U in f32 to caller scratch; a store kernel rounds it to bf16 back into
+//    the rows.  Both halves read every source row of a chunk before the store
+//    of that chunk starts (stream order), so the rotation is in place.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -143,14 +143,44 @@ cudaError_t launch_covariance_finalize(const float* C, int64_t c_s0, const float
   return cudaGetLastError();
 }
 
+namespace {
+
+// x U for rows [r0, r0 + n) of a uniformly strided row set (row r at
+// x + r * rs), into scratch [n, 512] f32: the V-up kernel with one "head"
+// whose rows are the requests, U's columns in two halves of 256.
+cudaError_t rotate_rows_f32(const __nv_bfloat16* x, int64_t rs, int64_t n, const void* U,
+                            float* scratch, cudaStream_t stream) {
+  const __nv_bfloat16* u = reinterpret_cast<const __nv_bfloat16*>(U);
+  for (int half = 0; half < 2; ++half) {
+    cudaError_t e = launch_vup(x, 1, rs, rs, u + 256 * half, (int64_t)kLatent * kLatent,
+                               kLatent, scratch + 256 * half, kLatent, kLatent, (int)n, 1, 256,
+                               stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
 cudaError_t launch_rotate(void* x, int64_t B, int64_t H, int64_t sb, int64_t sh, const void* U,
                           float* scratch, int64_t chunk_b, cudaStream_t stream) {
   __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(x);
+  const bool uniform = H == 1 || sb == H * sh;  // rows evenly spaced across b
+  const int64_t rs = H == 1 ? sb : sh;
+  // one V-up launch covers at most 65535 tiles of 64 rows
+  const int64_t max_rows = (int64_t)65535 * 64;
   for (int64_t b0 = 0; b0 < B; b0 += chunk_b) {
     const int64_t nb = B - b0 < chunk_b ? B - b0 : chunk_b;
-    // y[b, h, :] = x[b0 + b, h, :512] U, one U for every row (head stride 0)
-    cudaError_t e = launch_vup(xb + b0 * sb, 1, sb, sh, U, 0, kLatent, scratch, H * kLatent,
-                               kLatent, (int)nb, (int)H, kLatent, stream);
+    cudaError_t e = cudaSuccess;
+    if (uniform) {
+      for (int64_t r0 = 0; r0 < nb * H && e == cudaSuccess; r0 += max_rows) {
+        const int64_t n = nb * H - r0 < max_rows ? nb * H - r0 : max_rows;
+        e = rotate_rows_f32(xb + b0 * sb + r0 * rs, rs, n, U, scratch + r0 * kLatent, stream);
+      }
+    } else {
+      for (int64_t b = 0; b < nb && e == cudaSuccess; ++b)
+        e = rotate_rows_f32(xb + (b0 + b) * sb, sh, H, U, scratch + b * H * kLatent, stream);
+    }
     if (e != cudaSuccess) return e;
     const int64_t threads = nb * H * (kLatent / 8);
     const int64_t blocks = (threads + 255) / 256;

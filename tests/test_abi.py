@@ -282,3 +282,30 @@ def test_pca_entry_points_validate_without_launch():
     assert L.tpla_rotate_apply(B(rows), B(U), 0x20000, 64 * 512 * 4 - 16, None) == -4
     assert L.tpla_rotate_apply(B(rows), B(U), 0x20008, 1 << 20, None) == -4
     assert tp.launch_count() == before
+
+
+def test_cache_append_validates_without_launch():
+    L = tp.lib()
+    before = tp.launch_count()
+    B = ctypes.byref
+    new = _fake((3, 576), torch.bfloat16)
+    pos = _fake((3,), torch.int32)
+    pt = _fake((3, 4), torch.int32)
+    cache = _fake((10, 64, 576), torch.bfloat16)
+
+    def call(n=new, p=pos, t=pt, c=cache, groups=2, had=1, eps=1e-6):
+        return L.tpla_cache_append(B(n), B(p), B(t) if t is not None else None, B(c), groups,
+                                   had, ctypes.c_float(eps), None)
+
+    assert call(n=_fake((3, 512), torch.bfloat16)) == -1          # row width
+    assert call(n=_fake((3, 576), torch.int32)) == -1             # dtype
+    assert call(n=_fake((3, 576), torch.bfloat16, ptr=0x10002)) == -1  # alignment
+    assert call(p=_fake((2,), torch.int32)) == -1                 # one position per request
+    assert call(t=_fake((2, 4), torch.int32)) == -1               # page table rows
+    assert call(c=_fake((10, 32, 576), torch.bfloat16)) == -2     # 64-token pages only
+    assert call(c=_fake((10, 64, 576), torch.float32)) == -1      # bf16 cache
+    assert call(groups=3) == -1 and call(groups=16) == -1
+    assert call(had=2) == -1
+    assert call(eps=-1.0) == -1 and call(eps=float("nan")) == -1
+    assert call(t=None) == -1                                     # contiguous: [B, Lmax, 576]
+    assert tp.launch_count() == before

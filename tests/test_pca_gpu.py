@@ -21,7 +21,9 @@ def calib():
     w = make_inputs(4, 16, [4096, 4000, 64, 1000], paged=True, decay=True, seed=31, wuv=True)
     rows = as_f64(w.cache).reshape(-1, 576)
     lam, U = O.pca_basis_ref(rows[:, :512])
-    U16 = torch.from_numpy(U).to(torch.bfloat16)
+    # the eigensolver's basis comes back column-major; the library takes U
+    # row-major and contiguous
+    U16 = torch.from_numpy(np.ascontiguousarray(U)).to(torch.bfloat16)
     return w, rows, U16, as_f64(U16)
 
 
