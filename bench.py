@@ -47,7 +47,7 @@ NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (DGX figure); context beside the
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="dsv3", choices=sorted(CONFIGS))
@@ -56,7 +56,10 @@ def parse_args():
     ap.add_argument("--no-hadamard", action="store_true")
     ap.add_argument("--kernel", default="auto", choices=["auto", "generic", "sm100"])
     ap.add_argument("--num-splits", type=int, default=0)
-    ap.add_argument("--no-extras", action="store_true", help="skip the per-G sweep")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the per-G sweep and the other workloads")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (V2-Lite, Kimi-K2, long context)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--batch", type=int, default=None,
                     help="fewer requests of the same shape (profiling captures)")
@@ -505,7 +508,9 @@ def run_ours(args):
     t_tc = flops_step / (tc_peak * 1e12)
     used = "sm100" if args.kernel != "generic" and _sm100_used(tp, q, cache, seq, pt, G, rope, out,
                                                                 args) else "generic"
-    kname = "tpla_decode_sm100" if used == "sm100" else "decode_generic_kernel"
+    # G >= 2 runs the shard kernel (one CTA per TPLA shard), G = 1 the pair kernel
+    kname = (("tpla_decode_shard" if G >= 2 else "tpla_decode_sm100") if used == "sm100"
+             else "decode_generic_kernel")
     traffic = recorded_traffic(kname, args.config)
     if t_tc > t_hbm:
         roof = {"bound": "tensor", "achieved": round(achieved_tf, 2), "peak": tc_peak,
@@ -524,7 +529,11 @@ def run_ours(args):
 
     # ---- per-G decode-only sweep (vs G), full and one-shard
     vs_G = []
+    clk_extras = None
     if not args.no_extras:
+        cs = ClockSampler(local)
+        cs.start()
+        time.sleep(0.2)
         for GG, shard in ((1, None), (2, None), (4, None), (2, 0), (4, 0)):
             width = LATENT if shard is None else LATENT // GG
             o2 = torch.empty((B, H, width), dtype=torch.float32, device=dev)
@@ -533,7 +542,7 @@ def run_ours(args):
                 decode_once(q, o2, l2, shard, GG)
             a = torch.cuda.Event(enable_timing=True)
             bb = torch.cuda.Event(enable_timing=True)
-            n = 10
+            n = 50
             a.record(stream)
             for _ in range(n):
                 decode_once(q, o2, l2, shard, GG)
@@ -547,6 +556,13 @@ def run_ours(args):
                          "hbm_frac": round(nb / t / 1e9 / hbm_peak, 4),
                          "tok_s_layer": round(B / t, 1)})
             del o2, l2
+        clk_extras = cs.stop()
+
+    configs = None
+    if not args.no_extras and not args.no_configs and world == 1:
+        del cache, q, ws, out, y
+        torch.cuda.empty_cache()
+        configs = other_workloads(tp, dev, hbm_peak, tc_peak)
 
     cpu = None
     if rank == 0 and world == 1:
@@ -570,7 +586,9 @@ def run_ours(args):
         "config": step_config(args, w, used, f"replicas x{world}"),
         "tok_s_layer": round(tok_s, 1),
         "hbm_frac_step": round(value / world / hbm_peak, 4),
-        "roofline": roof, "vs_G": vs_G, "one_shard_speedup_vs_mla": one_shard_speedups(vs_G),
+        "roofline": roof, "vs_G": vs_G, "vs_G_clocks": clk_extras,
+        "one_shard_speedup_vs_mla": one_shard_speedups(vs_G),
+        "configs": configs,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "pipelining": "H2D, compute and D2H on three streams, two buffer sets",
@@ -580,6 +598,108 @@ def run_ours(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def other_workloads(tp, dev, hbm_peak, tc_peak):
+    """Decode (and V-up) timings of the other configured workloads, each on
+    its own seeded inputs with the Hadamard reparameterisation folded in:
+    DeepSeek-V2-Lite shape (G=2), Kimi-K2 shape (G=1/2/4, both rope modes,
+    V-up combine), long context (B=4, 131072 tokens; automatic split against
+    32/64/128 explicit chunks, G=1/4).  A cache smaller than twice the L2 is
+    timed launch by launch with the L2 flushed in between (a 256 MB write
+    outside the timed events); the others stream more than L2 holds."""
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    plan = {
+        "v2lite": [dict(G=2, rope="replicate", splits=0, vup=True)],
+        "kimi": [dict(G=G, rope=r, splits=0, vup=True) for G in (1, 2, 4)
+                 for r in ("replicate", "split")],
+        "long": [dict(G=G, rope="replicate", splits=sp, vup=False) for G in (1, 4)
+                 for sp in (0, 32, 64, 128)],
+    }
+    res = {}
+    for name, settings in plan.items():
+        w = make_workload(name)
+        q = w.q.to(dev)
+        cache = w.cache.to(dev)
+        seq = w.seq_lens.to(dev)
+        pt = None if w.page_table is None else w.page_table.to(dev)
+        tp.hadamard_apply(q, LATENT)
+        tp.hadamard_apply(cache, LATENT)
+        W = None
+        if w.W_uv is not None:
+            Wt = w.W_uv.to(dev).transpose(1, 2).contiguous()
+            tp.hadamard_apply(Wt, LATENT)
+            W = Wt.transpose(1, 2).contiguous()
+        small = cache.numel() * 2 < 2 * L2_BYTES
+        tokens = int(w.seq_lens.to(torch.int64).sum())
+        cs = ClockSampler(dev.index or 0)
+        cs.start()
+        time.sleep(0.2)
+        rows = []
+        for st in settings:
+            G, rope = st["G"], st["rope"]
+            out = torch.empty((w.B, w.H, LATENT), dtype=torch.float32, device=dev)
+            lse = torch.empty((w.B, w.H, G), dtype=torch.float32, device=dev)
+            y = torch.empty((w.B, w.H, 128), dtype=torch.float32, device=dev)
+            need = tp.decode_workspace_size(q, cache, seq, pt, G, rope, out, num_splits=st["splits"])
+            ws = torch.empty(max(16, need), dtype=torch.uint8, device=dev)
+
+            def dec():
+                tp.decode(q, cache, seq, pt, G, rope, w.scale, out=out, lse=lse,
+                          num_splits=st["splits"], workspace=ws)
+
+            def timed(fn, n):
+                ts = []
+                for _ in range(3):
+                    fn()
+                for i in range(n):
+                    if small or i == 0:
+                        flush.zero_()
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    fn()
+                    b.record()
+                    if small:
+                        torch.cuda.synchronize()
+                        ts.append(a.elapsed_time(b))
+                    else:
+                        ts.append((a, b))
+                torch.cuda.synchronize()
+                if not small:
+                    ts = [x.elapsed_time(z) for x, z in ts]
+                return statistics.median(ts) / 1e3
+
+            t = timed(dec, 50)
+            nb = w.latent_kv_bytes(G, None, rope)
+            fl = tokens * w.H * flops_per_token_head(G, None, rope)
+            t_roof = max(nb / (hbm_peak * 1e9), fl / (tc_peak * 1e12))
+            row = {"G": G, "rope": rope, "splits": st["splits"] or "auto",
+                   "decode_us": round(t * 1e6, 1), "GB_s": round(nb / t / 1e9, 1),
+                   "hbm_frac": round(nb / t / 1e9 / hbm_peak, 4),
+                   "tensor_tflops": round(fl / t / 1e12, 1),
+                   "roofline_frac": round(t_roof / t, 4),
+                   "tok_s_layer": round(w.B / t, 1)}
+            if st["vup"] and W is not None:
+                tv = timed(lambda: tp.vup_combine(out, W, y), 50)
+                vb = out.numel() * 4 + W.numel() * 2 + y.numel() * 4
+                row.update({"vup_us": round(tv * 1e6, 2),
+                            "vup_hbm_frac": round(vb / tv / 1e9 / hbm_peak, 4),
+                            "step_us": round((t + tv) * 1e6, 1)})
+            rows.append(row)
+            del out, lse, y, ws
+        res[name] = {"B": w.B, "H": w.H, "tokens": tokens,
+                     "cache_bytes": int(cache.numel() * 2),
+                     "timing": "median of 50 launches, L2 flushed before each" if small
+                               else "median of 50 back-to-back launches (cache > 2x L2)",
+                     "rows": rows, "clocks": cs.stop()}
+        del q, cache, seq, pt, W
+        torch.cuda.empty_cache()
+    del flush
+    return res
 
 
 def _sm100_used(tp, q, cache, seq, pt, G, rope, out, args):
