@@ -1477,13 +1477,11 @@ sm100_merge_kernel(const Params p) {
     }
     return;
   }
-  auto slot_of = [&](int c) -> int {
-    if (p.mode == 0) {
-      const long long start = (long long)c * T / P;
-      return (c == s_lo && start < pre) ? 2 * c + 1 : 2 * c;
-    }
-    return 2 * c;
-  };
+  // Slot of range c's partial of this request: 2c, except the first range,
+  // which used its second slot when the request started inside it (the one
+  // 64-bit division is done once here).
+  const int first_slot = (p.mode == 0 && (long long)s_lo * T / P < pre) ? 2 * s_lo + 1 : 2 * s_lo;
+  auto slot_of = [&](int c) -> int { return c == s_lo ? first_slot : 2 * c; };
   // Column groups of this lane: 16-byte groups 4 * lane + 128 * i of each
   // shard (cw <= 512, so at most four).  Loads of two slots x all groups go
   // out together before the multiply-adds.
@@ -1494,15 +1492,20 @@ sm100_merge_kernel(const Params p) {
       return reinterpret_cast<const float4*>(p.part_o + ((int64_t)slot_of(c) * p.H + h) * p.W +
                                              k * cw) + lane;
     };
-    float M = -INFINITY;
-    for (int c = s_lo + lane; c <= s_hi; c += 32) M = fmaxf(M, lse_of(c));
+    // lane i holds the lse of slot s_lo + i (the first 32 slots; the usual
+    // case has two)
+    const float ls_lane = s_lo + lane <= s_hi ? lse_of(s_lo + lane) : -INFINITY;
+    float M = ls_lane;
+    for (int c = s_lo + 32 + lane; c <= s_hi; c += 32) M = fmaxf(M, lse_of(c));
     M = warp_max(M);
     float z = 0.f;
-    if (M != -INFINITY)
-      for (int c = s_lo + lane; c <= s_hi; c += 32) {
+    if (M != -INFINITY) {
+      z = ls_lane == -INFINITY ? 0.f : expf(ls_lane - M);
+      for (int c = s_lo + 32 + lane; c <= s_hi; c += 32) {
         const float ls = lse_of(c);
         z += ls == -INFINITY ? 0.f : expf(ls - M);
       }
+    }
     z = warp_sum(z);
     const float total = M == -INFINITY ? -INFINITY : M + logf(z);
     float4 acc[4];
@@ -1510,11 +1513,8 @@ sm100_merge_kernel(const Params p) {
     for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (total != -INFINITY) {
       for (int g0 = s_lo; g0 <= s_hi; g0 += 32) {
-        float wmine = 0.f;
-        if (g0 + lane <= s_hi) {
-          const float ls = lse_of(g0 + lane);
-          wmine = ls == -INFINITY ? 0.f : expf(ls - total);
-        }
+        const float lsm = g0 == s_lo ? ls_lane : (g0 + lane <= s_hi ? lse_of(g0 + lane) : -INFINITY);
+        const float wmine = lsm == -INFINITY ? 0.f : expf(lsm - total);
         const int n = min(32, s_hi - g0 + 1);
         for (int i0 = 0; i0 < n; i0 += 2) {
           const float w0 = __shfl_sync(0xffffffffu, wmine, i0);
