@@ -58,6 +58,15 @@ Readings taken where the pages are silent:
    taken over each of ``norm_groups`` contiguous shards (one group: exact
    MLA; G groups: every TPLA rank normalises its own slice).  The rotation,
    when used, comes first; eps is added to the mean square.
+11. Prefill/decode separation ([ABSTRACT]: MLA-style prefilling, then
+   tensor-parallel decoding; [REVIEW referee_report.major_comments] on Table
+   2: the separated variant runs unmodified MLA during prefill and TPLA only
+   during decode).  The prefill of a request stores its prompt rows through
+   the cache-write step of reading 10 and gives every prompt token the exact
+   MLA attention (one softmax over all 576 values per token) over the
+   request's stored rows up to and including its own position (causal).  It
+   is written in the absorbed form the decode uses; the per-head
+   up-projected form of MLA is the same function in exact arithmetic.
 """
 
 from __future__ import annotations
@@ -493,6 +502,30 @@ def cache_append_ref(cache, kv_new, positions, page_table, norm_groups, hadamard
         else:
             out[np.asarray(page_table)[b][pos // BLOCK], pos % BLOCK] = rows[b]
     return out
+
+
+def mla_prefill_ref(q, rows, start, scale):
+    """Exact MLA over a request's prompt tokens, causally (reading 11).
+
+    Prompt token i sits at position start + i and attends, with one softmax
+    over all 576 values per token as in ``mla_decode_ref``, to the request's
+    stored rows 0 .. start + i: the rows cached before the prompt and the
+    prompt's own rows up to and including itself.
+    q [T, H, 576] (absorbed queries of the prompt tokens); rows
+    [>= start + T, 576] (the request's stored rows, in position order).
+    Returns out [T, H, 512] and lse [T, H].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    rows = np.asarray(rows, dtype=np.float64)
+    T, H, _ = q.shape
+    if start < 0 or rows.shape[0] < start + T:
+        raise ValueError("rows must hold the prefix and every prompt token")
+    out = np.zeros((T, H, LATENT))
+    lse = np.zeros((T, H))
+    for i in range(T):
+        c = rows[:start + i + 1]
+        out[i], lse[i] = attention_ref(q[i], c, c[:, :LATENT], scale)
+    return out, lse
 
 
 # ---------------------------------------------------------------------------

@@ -668,3 +668,82 @@ def test_cache_append_pins_catch_planted_mistakes(monkeypatch):
         want = _cache_row_bruteforce(a, 4, False, 1e-6)
         assert np.abs(got - np.asarray(want)).max() > 1e-3, bad.__name__
     monkeypatch.setattr(O, "rms_norm_groups_ref", good)
+
+
+# ---------------------------------------------------------------- prefill (exact MLA, causal)
+
+def _masked_prefill(q, rows, start, scale):
+    """Causal attention written as one score matrix over all stored rows with
+    the positions after each query masked to -inf (the mask form, not the
+    prefix slices the oracle takes)."""
+    T, H, _ = q.shape
+    n = start + T
+    out = np.zeros((T, H, O.LATENT))
+    lse = np.zeros((T, H))
+    for i in range(T):
+        for h in range(H):
+            s = np.array([scale * math.fsum(float(a) * float(b) for a, b in zip(q[i, h], rows[t]))
+                          for t in range(n)])
+            s[np.arange(n) > start + i] = -np.inf
+            m = s.max()
+            w = np.exp(s - m)
+            z = math.fsum(w)
+            out[i, h] = (w[:, None] * rows[:n, :O.LATENT]).sum(0) / z
+            lse[i, h] = m + math.log(z)
+    return out, lse
+
+
+@pytest.mark.parametrize("start", [0, 3])
+def test_prefill_matches_masked_bruteforce(start):
+    T, H = 4, 2
+    q = _rand((T, H, O.WIDTH), 40 + start)
+    rows = _rand((start + T, O.WIDTH), 50 + start)
+    got_o, got_l = O.mla_prefill_ref(q, rows, start, SCALE)
+    want_o, want_l = _masked_prefill(q, rows, start, SCALE)
+    np.testing.assert_allclose(got_o, want_o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(got_l, want_l, rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_first_token_closed_form():
+    """With nothing cached, prompt token 0 sees only its own row: the output
+    is that row's latent and lse its own score."""
+    q = _rand((3, 4, O.WIDTH), 61)
+    rows = _rand((3, O.WIDTH), 62)
+    out, lse = O.mla_prefill_ref(q, rows, 0, SCALE)
+    np.testing.assert_allclose(out[0], np.broadcast_to(rows[0, :O.LATENT], (4, O.LATENT)),
+                               rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse[0], SCALE * (q[0] @ rows[0]), rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_last_token_is_a_decode_and_causal():
+    start, T, H = 5, 6, 3
+    q = _rand((T, H, O.WIDTH), 63)
+    rows = _rand((start + T, O.WIDTH), 64)
+    out, lse = O.mla_prefill_ref(q, rows, start, SCALE)
+    # the last prompt token attends to the whole request: one decode step
+    do, dl = O.mla_decode_ref(q[-1:], [rows], SCALE)
+    np.testing.assert_allclose(out[-1], do[0], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse[-1], dl[0], rtol=1e-12, atol=1e-12)
+    # rows after position start + i never reach token i; they do reach later ones
+    other = rows.copy()
+    other[start + 3:] += 1.0
+    out2, _ = O.mla_prefill_ref(q, other, start, SCALE)
+    np.testing.assert_array_equal(out2[:3], out[:3])
+    assert np.abs(out2[3:] - out[3:]).max() > 1e-3
+
+
+def test_prefill_pins_catch_planted_mistakes(monkeypatch):
+    """An off-by-one prefix (token i seeing only rows before it) fails the
+    closed form and the masked brute force."""
+    good = O.attention_ref
+    q = _rand((3, 2, O.WIDTH), 65)
+    rows = _rand((3, O.WIDTH), 66)
+
+    def shifted(qh, keys, values, scale):  # drops the token's own row
+        return good(qh, keys[:-1], values[:-1], scale)
+
+    monkeypatch.setattr(O, "attention_ref", shifted)
+    out, _ = O.mla_prefill_ref(q, rows, 0, SCALE)
+    assert not np.allclose(out[0], rows[0, :O.LATENT])
+    want, _ = _masked_prefill(q, rows, 0, SCALE)
+    assert not np.allclose(out, want)
