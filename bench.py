@@ -563,6 +563,7 @@ def run_ours(args):
         del cache, q, ws, out, y
         torch.cuda.empty_cache()
         configs = other_workloads(tp, dev, hbm_peak, tc_peak)
+        configs["prefill"] = prefill_workload(tp, dev, tc_peak)
 
     cpu = None
     if rank == 0 and world == 1:
@@ -699,6 +700,54 @@ def other_workloads(tp, dev, hbm_peak, tc_peak):
         del q, cache, seq, pt, W
         torch.cuda.empty_cache()
     del flush
+    return res
+
+
+def prefill_workload(tp, dev, tc_peak):
+    """Prefill of one DeepSeek-V3-shaped request (H = 128) under prefill/decode
+    separation: the prompt rows into the paged cache, then exact MLA (G = 1)
+    of every prompt token over its causal prefix (tpla_prefill).  FLOPs are
+    the absorbed form's 2176 per (query token, cached token, head) over the
+    causal pairs; the prompt's cache (T x 1152 B) stays in L2, so the bound is
+    the tensor pipe.  Median of 10 calls after 3 warm-up calls."""
+    from mla_latent_kv_dim_b200.workloads import make_prefill_inputs
+    res = {"rows": [], "timing": "median of 10 calls (append + attention + merge)"}
+    cs = ClockSampler(dev.index or 0)
+    cs.start()
+    time.sleep(0.2)
+    for T in (4096, 16384):
+        w = make_prefill_inputs(T, 128, 0, seed=31)
+        q, new = w.q.to(dev), w.kv_new.to(dev)
+        row, cache = w.page_row.to(dev), w.cache.to(dev)
+        out = torch.empty((T, 128, LATENT), dtype=torch.float32, device=dev)
+        lse = torch.empty((T, 128, 1), dtype=torch.float32, device=dev)
+        ws = torch.empty(1 << 24, dtype=torch.uint8, device=dev)
+
+        def call():
+            tp.prefill(q, new, 0, row, cache, scale=w.scale, out=out, lse=lse, workspace=ws)
+
+        for _ in range(3):
+            call()
+        ts = []
+        for _ in range(10):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        t = statistics.median([x.elapsed_time(z) for x, z in ts]) / 1e3
+        pairs = T * (T + 1) // 2
+        fl = pairs * 128 * flops_per_token_head(1)
+        res["rows"].append({"T": T, "H": 128, "causal_pairs": pairs,
+                            "prefill_us": round(t * 1e6, 1),
+                            "tensor_tflops": round(fl / t / 1e12, 1),
+                            "tensor_frac": round(fl / t / 1e12 / tc_peak, 4),
+                            "prompt_tok_s": round(T / t, 1)})
+        del q, new, row, cache, out, lse, ws
+        torch.cuda.empty_cache()
+    res["clocks"] = cs.stop()
     return res
 
 

@@ -323,6 +323,57 @@ TPLA_API int tpla_cache_append(const tpla_tensor* kv_new, const tpla_tensor* pos
                                int norm_groups, int hadamard, float eps,
                                tpla_stream_t stream);
 
+/*
+ * tpla_prefill -- the prefill half of prefill/decode separation, for T prompt
+ * tokens of one request.  The TPLA abstract: models pre-trained with MLA keep
+ * MLA-style prefilling and decode tensor-parallel; the TPLA review (referee
+ * report, major comment on Table 2 and the abstract; forward implications):
+ * the separated variant runs exact MLA in the compute-bound prefill and TPLA
+ * only in decode.  Two steps, in stream order on `stream`:
+ *  1. row i of kv_new is stored at position start + i of the request,
+ *     exactly as tpla_cache_append stores a row (optional Hadamard rotation,
+ *     RMS norm over norm_groups slices, one bf16 rounding);
+ *  2. prompt token i gets exact MLA attention -- one softmax over all 576
+ *     values of each token, absorbed form, G = 1 -- over the request's stored
+ *     rows 0 .. start + i (causal): out[i] and lse[i].  The tcgen05 kernel of
+ *     tpla_decode_ex runs it with one query row per prompt token, the
+ *     lengths start + i + 1 computed in the kernel and the page-table row
+ *     shared by every query row; the split-KV merge follows.
+ * A later tpla_decode_ex of the request (any G) reads the same stored rows.
+ *   q         [T, H, 576] bf16: the prompt tokens' absorbed queries (the
+ *             layout of tpla_decode_ex's q; 16-byte aligned rows).
+ *   kv_new    [T, 576] bf16 or f32: tpla_cache_append's row layout.
+ *   start     >= 0: tokens of the request already in the cache.
+ *   page_row  [max_pages] int32, contiguous: the request's page-table row;
+ *             start + T <= 64 * max_pages.  Page ids must lie in
+ *             [0, num_blocks): others are not written or read, and the
+ *             kernels record TPLA_ERR_DEVICE_BOUNDS.
+ *   kv_cache  [num_blocks, 64, 576] bf16, the paged layout (16-byte aligned
+ *             rows); updated in place.
+ *   norm_groups, hadamard, eps: as in tpla_cache_append.
+ *   scale     softmax scale, any finite value (as in tpla_decode_ex).
+ *   out       [T, H, 512] f32 or bf16 (16-byte aligned rows); lse [T, H, 1]
+ *             f32 or NULL.
+ *   workspace split scratch of at least tpla_prefill_workspace_size bytes,
+ *             16-byte aligned, or NULL: the call then takes it from the
+ *             stream-ordered allocator (cudaMallocAsync / cudaFreeAsync on
+ *             `stream`), as tpla_decode does.
+ * Errors before any launch: TPLA_ERR_INVALID_ARG (shapes, dtypes, strides,
+ * alignment, start, a page row too short for start + T, norm_groups,
+ * hadamard, eps, scale); TPLA_ERR_UNSUPPORTED (T > 2^20, H > 4096,
+ * T * H > 2^30, pages other than 64 tokens, no sm_100 GPU);
+ * TPLA_ERR_WORKSPACE (a workspace that is short or misaligned).
+ */
+TPLA_API int tpla_prefill(const tpla_tensor* q, const tpla_tensor* kv_new, int start,
+                          const tpla_tensor* page_row, tpla_tensor* kv_cache, int norm_groups,
+                          int hadamard, float eps, float scale, tpla_tensor* out,
+                          tpla_tensor* lse, void* workspace, size_t workspace_bytes,
+                          tpla_stream_t stream);
+
+/* tpla_prefill_workspace_size -- bytes of workspace tpla_prefill needs for
+ * queries q ([T, H, 576] bf16) on the current device. */
+TPLA_API int tpla_prefill_workspace_size(const tpla_tensor* q, size_t* bytes);
+
 /* Human-readable name of a tpla_status code (static string). */
 TPLA_API const char* tpla_error_string(int status);
 

@@ -8,9 +8,10 @@ workloads (``workloads``).
 from ._native import (TplaError, cache_append, decode, decode_simple,  # noqa: F401
                       decode_workspace_size,
                       device_status, error_string, hadamard_apply, latent_covariance,
-                      launch_count, lse_merge, lib, rotate_apply, selftest_wait_timeout,
-                      version, vup_combine)
+                      launch_count, lse_merge, lib, prefill, rotate_apply,
+                      selftest_wait_timeout, version, vup_combine)
 
 __all__ = ["TplaError", "cache_append", "decode", "decode_simple", "decode_workspace_size", "device_status",
            "selftest_wait_timeout", "latent_covariance", "rotate_apply",
-           "error_string", "hadamard_apply", "launch_count", "lse_merge", "lib", "version", "vup_combine"]
+           "error_string", "hadamard_apply", "launch_count", "lse_merge", "lib", "prefill", "version",
+           "vup_combine"]

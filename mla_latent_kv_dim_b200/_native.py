@@ -82,11 +82,16 @@ def lib() -> ctypes.CDLL:
                                             ctypes.c_void_p]
             L.tpla_cache_append.argtypes = [T, T, T, T, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_float, ctypes.c_void_p]
+            L.tpla_prefill.argtypes = [T, T, ctypes.c_int, T, T, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_float, ctypes.c_float, T, T, ctypes.c_void_p,
+                                       ctypes.c_size_t, ctypes.c_void_p]
+            L.tpla_prefill_workspace_size.argtypes = [T, _P(ctypes.c_size_t)]
             for f in ("tpla_decode_ex", "tpla_decode", "tpla_decode_workspace_size",
                       "tpla_lse_merge", "tpla_hadamard_apply", "tpla_vup_combine",
                       "tpla_last_cuda_error", "tpla_get_device_status", "tpla_version",
                       "tpla_selftest_wait_timeout", "tpla_latent_covariance",
-                      "tpla_covariance_finalize", "tpla_rotate_apply", "tpla_cache_append"):
+                      "tpla_covariance_finalize", "tpla_rotate_apply", "tpla_cache_append",
+                      "tpla_prefill", "tpla_prefill_workspace_size"):
                 getattr(L, f).restype = ctypes.c_int
             L.tpla_launch_count.restype = ctypes.c_int64
             _lib = L
@@ -297,6 +302,38 @@ def cache_append(kv_new, positions, page_table, kv_cache, norm_groups=1, hadamar
                                  ctypes.c_float(eps), _stream(stream))
     _check("tpla_cache_append", rc)
     return kv_cache
+
+
+def prefill(q, kv_new, start, page_row, kv_cache, norm_groups=1, hadamard=False, eps=1e-6,
+            scale=None, out=None, lse=None, *, workspace=None, out_dtype=torch.float32,
+            want_lse=True, stream=None):
+    """Prefill of one request (tpla_prefill): store the prompt rows ``kv_new``
+    [T, 576] at positions start .. start + T - 1 through the request's page
+    row ``page_row`` [max_pages] (as ``cache_append`` stores a row), then exact
+    MLA of every prompt token (``q`` [T, H, 576]) over its causal prefix.
+    Returns (out [T, H, 512], lse [T, H, 1]); ``kv_cache`` is updated in
+    place."""
+    if scale is None:
+        raise ValueError("scale is required")
+    _on_current_device(q, kv_new, page_row, kv_cache, out, lse, workspace)
+    T, H = q.shape[0], q.shape[1]
+    if out is None:
+        out = torch.empty((T, H, 512), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((T, H, 1), dtype=torch.float32, device=q.device)
+    n = ctypes.c_size_t(0)
+    _check("tpla_prefill_workspace_size",
+           lib().tpla_prefill_workspace_size(_ref(desc(q)), ctypes.byref(n)))
+    need = int(n.value)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty((need + 15) // 16 * 16, dtype=torch.uint8, device=q.device)
+    rc = lib().tpla_prefill(
+        _ref(desc(q)), _ref(desc(kv_new)), int(start), _ref(desc(page_row)), _ref(desc(kv_cache)),
+        int(norm_groups), 1 if hadamard else 0, ctypes.c_float(eps), ctypes.c_float(scale),
+        _ref(desc(out)), _ref(desc(lse)), workspace.data_ptr() if need else None,
+        workspace.numel() * workspace.element_size() if need else 0, _stream(stream))
+    _check("tpla_prefill", rc)
+    return out, lse
 
 
 def device_status(stream=None) -> int:

@@ -194,6 +194,77 @@ int run_decode(const DecodeProblem& p, const tpla_decode_opts* opts, Path path, 
   return TPLA_OK;
 }
 
+// A validated prefill call: the exact-MLA attention of its prompt rows as a
+// decode problem with one query row per prompt token, causal lengths and the
+// request's page-table row shared by every query row (row stride 0).
+struct PrefillCall {
+  DecodeProblem p;
+};
+
+int build_prefill(const tpla_tensor* q, const tpla_tensor* kv_new, int start,
+                  const tpla_tensor* page_row, const tpla_tensor* kv, int norm_groups,
+                  int hadamard, float eps, float scale, const tpla_tensor* out,
+                  const tpla_tensor* lse, PrefillCall* c) {
+  memset(c, 0, sizeof(*c));
+  if (!check_tensor(q, TPLA_BF16, 3) || q->shape[2] != kWidth) return TPLA_ERR_INVALID_ARG;
+  const int64_t T = q->shape[0], H = q->shape[1];
+  if (T > (1 << 20) || H > 4096) return TPLA_ERR_UNSUPPORTED;
+  if (T * H > kMaxRequestHeads) return TPLA_ERR_UNSUPPORTED;
+  if (T > 0 && H > 0 && (!aligned16(q->data) || (q->stride[1] % 8) || (q->stride[0] % 8)))
+    return TPLA_ERR_INVALID_ARG;
+  c->p.B = (int)T;
+  c->p.H = (int)H;
+  c->p.G = 1;
+  c->p.shard = -1;
+  c->p.n_shards = 1;
+  c->p.out_width = kLatent;
+  if (!kv_new) return TPLA_OK;  // workspace-size query: q alone fixes it
+  if (kv_new->dtype != TPLA_BF16 && kv_new->dtype != TPLA_F32) return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(kv_new, kv_new->dtype, 2) || kv_new->shape[0] != T ||
+      kv_new->shape[1] != kWidth)
+    return TPLA_ERR_INVALID_ARG;
+  const int64_t esz = kv_new->dtype == TPLA_BF16 ? 2 : 4;
+  if (T > 0 && (!aligned16(kv_new->data) || (kv_new->stride[0] * esz) % 16))
+    return TPLA_ERR_INVALID_ARG;
+  if (start < 0) return TPLA_ERR_INVALID_ARG;
+  if (!(norm_groups == 1 || norm_groups == 2 || norm_groups == 4 || norm_groups == 8))
+    return TPLA_ERR_INVALID_ARG;
+  if (!(hadamard == 0 || hadamard == 1) || !isfinite(eps) || eps < 0.f)
+    return TPLA_ERR_INVALID_ARG;
+  if (!kv || !check_tensor(kv, TPLA_BF16, 3) || kv->shape[2] != kWidth)
+    return TPLA_ERR_INVALID_ARG;
+  if (kv->shape[1] != kBlock) return TPLA_ERR_UNSUPPORTED;  // 64-token pages only
+  if (!aligned16(kv->data) || kv->stride[0] % 8 || kv->stride[1] % 8)
+    return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(page_row, TPLA_I32, 1) || page_row->shape[0] < 1) return TPLA_ERR_INVALID_ARG;
+  if (page_row->shape[0] > (1 << 24)) return TPLA_ERR_UNSUPPORTED;
+  if ((int64_t)start + T > page_row->shape[0] * kBlock) return TPLA_ERR_INVALID_ARG;
+  // the attention half is a decode problem: query row i holds start + i + 1
+  // tokens, every row reads the request's page-table row
+  tpla_tensor pt = *page_row;
+  pt.ndim = 2;
+  pt.shape[0] = T;
+  pt.shape[1] = page_row->shape[0];
+  pt.stride[0] = 0;
+  pt.stride[1] = 1;
+  int placeholder = 0;  // stands for a lengths array that is never read
+  tpla_tensor seq;
+  memset(&seq, 0, sizeof(seq));
+  seq.data = &placeholder;
+  seq.dtype = TPLA_I32;
+  seq.ndim = 1;
+  seq.shape[0] = T;
+  seq.stride[0] = 1;
+  int rc = build_problem(q, kv, &seq, &pt, 1, TPLA_ROPE_REPLICATE, scale, out, lse, nullptr,
+                         &c->p);
+  if (rc != TPLA_OK) return rc;
+  c->p.seq_lens = nullptr;
+  c->p.causal_base = start;
+  if (c->p.B > 0 && c->p.H > 0 && !sm100_supported(c->p, current_device()))
+    return TPLA_ERR_UNSUPPORTED;
+  return TPLA_OK;
+}
+
 }  // namespace
 
 void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
@@ -438,12 +509,59 @@ int tpla_cache_append(const tpla_tensor* kv_new, const tpla_tensor* positions,
   if (B == 0) return TPLA_OK;
   cudaError_t e = launch_cache_append(
       kv_new->data, kv_new->dtype == TPLA_BF16, kv_new->stride[0],
-      reinterpret_cast<const int*>(positions->data),
+      reinterpret_cast<const int*>(positions->data), 0,
       page_table ? reinterpret_cast<const int*>(page_table->data) : nullptr,
       page_table ? page_table->stride[0] : 0, max_pages, kv_cache->shape[0], kv_cache->shape[1],
       kv_cache->data, kv_cache->stride[0], kv_cache->stride[1], (int)B, norm_groups, hadamard,
       eps, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
+}
+
+int tpla_prefill_workspace_size(const tpla_tensor* q, size_t* bytes) {
+  if (!bytes) return TPLA_ERR_INVALID_ARG;
+  PrefillCall c;
+  int rc = build_prefill(q, nullptr, 0, nullptr, nullptr, 1, 0, 0.f, 1.0f, nullptr, nullptr, &c);
+  if (rc != TPLA_OK) return rc;
+  *bytes = c.p.H > 0 ? sm100_workspace_bytes(c.p, 0, current_device()) : 0;
+  return TPLA_OK;
+}
+
+int tpla_prefill(const tpla_tensor* q, const tpla_tensor* kv_new, int start,
+                 const tpla_tensor* page_row, tpla_tensor* kv_cache, int norm_groups,
+                 int hadamard, float eps, float scale, tpla_tensor* out, tpla_tensor* lse,
+                 void* workspace, size_t workspace_bytes, tpla_stream_t stream) {
+  PrefillCall c;
+  int rc = build_prefill(q, kv_new, start, page_row, kv_cache, norm_groups, hadamard, eps, scale,
+                         out, lse, &c);
+  if (rc != TPLA_OK) return rc;
+  const DecodeProblem& p = c.p;
+  if (p.B == 0) return TPLA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  size_t need = p.H > 0 ? sm100_workspace_bytes(p, 0, current_device()) : 0;
+  if (workspace && (workspace_bytes < need || !aligned16(workspace))) return TPLA_ERR_WORKSPACE;
+  // 1. the prompt rows into the cache (row b at position start + b)
+  cudaError_t e = launch_cache_append(
+      kv_new->data, kv_new->dtype == TPLA_BF16, kv_new->stride[0], nullptr, start,
+      reinterpret_cast<const int*>(page_row->data), 0, (int)page_row->shape[0],
+      kv_cache->shape[0], 0, kv_cache->data, kv_cache->stride[0], kv_cache->stride[1], p.B,
+      norm_groups, hadamard, eps, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (p.H == 0) return TPLA_OK;
+  // 2. exact MLA of every prompt token over its causal prefix
+  void* ws = workspace;
+  bool owned = false;
+  if (!ws && need > 0) {
+    e = cudaMallocAsync(&ws, need, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    owned = true;
+  }
+  e = launch_decode_sm100(p, 0, ws, need, s);
+  rc = e == cudaSuccess ? TPLA_OK : cuda_fail(e);
+  if (owned) {
+    e = cudaFreeAsync(ws, s);
+    if (rc == TPLA_OK && e != cudaSuccess) rc = cuda_fail(e);
+  }
+  return rc;
 }
 
 const char* tpla_error_string(int status) {

@@ -38,7 +38,8 @@ struct AppendParams {
   const void* kv_new;
   int in_bf16;
   int64_t n_sb;
-  const int* positions;
+  const int* positions;  // nullptr: row b goes to position pos0 + b
+  int pos0;
   const int* page_table;
   int64_t pt_sb;
   int max_pages;
@@ -57,7 +58,7 @@ __global__ void __launch_bounds__(kWarps * 32) cache_append_kernel(const AppendP
   const int b = blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (b >= p.B) return;
   // destination row
-  const int pos = p.positions[b];
+  const int pos = p.positions ? p.positions[b] : p.pos0 + b;
   __nv_bfloat16* dst = nullptr;
   if (p.page_table) {
     if (pos >= 0 && pos < 64 * p.max_pages) {
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(kWarps * 32) cache_append_kernel(const AppendP
 }  // namespace
 
 cudaError_t launch_cache_append(const void* kv_new, int in_bf16, int64_t n_sb, const int* positions,
-                                const int* page_table, int64_t pt_sb, int max_pages,
+                                int pos0, const int* page_table, int64_t pt_sb, int max_pages,
                                 int64_t num_blocks, int64_t cap_rows, void* cache, int64_t c_s0,
                                 int64_t c_s1, int B, int groups, int hadamard, float eps,
                                 cudaStream_t stream) {
@@ -160,6 +161,7 @@ cudaError_t launch_cache_append(const void* kv_new, int in_bf16, int64_t n_sb, c
   p.in_bf16 = in_bf16;
   p.n_sb = n_sb;
   p.positions = positions;
+  p.pos0 = pos0;
   p.page_table = page_table;
   p.pt_sb = pt_sb;
   p.max_pages = max_pages;

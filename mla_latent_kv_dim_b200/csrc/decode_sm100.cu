@@ -112,7 +112,8 @@ __device__ int g_status;
 __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
 
 struct Params {
-  const int* seq_lens;
+  const int* seq_lens;  // [B], or nullptr: request b holds causal_base + b + 1 tokens
+  int causal_base;      // (the query rows of a prompt, each seeing its causal prefix)
   const int* page_table;
   int64_t pt_sb;
   int num_blocks;   // paged: physical blocks (block index num_blocks reads as zeros)
@@ -143,7 +144,7 @@ struct Params {
 // ---------------------------------------------------------------- schedule
 
 __device__ __forceinline__ int req_len(const Params& p, int b) {
-  int L = p.seq_lens[b];
+  int L = p.seq_lens ? p.seq_lens[b] : p.causal_base + b + 1;
   if (L < 0 || L > p.cap_tokens) {
     set_status(TPLA_ERR_DEVICE_BOUNDS);
     L = L < 0 ? 0 : p.cap_tokens;
@@ -153,6 +154,23 @@ __device__ __forceinline__ int req_len(const Params& p, int b) {
 
 __device__ __forceinline__ int req_tiles(const Params& p, int b) {
   return (req_len(p, b) + p.tile_tok - 1) / p.tile_tok;
+}
+
+// Causal lengths: sum over n = 1 .. N of ceil(n / tile_tok), in closed form.
+__device__ __forceinline__ long long causal_tile_sum(const Params& p, long long N) {
+  const long long tt = p.tile_tok, q = N / tt, r = N % tt;
+  return tt * q * (q + 1) / 2 + r * (q + 1);
+}
+
+// Tiles of requests [0, b).  Lengths from seq_lens are summed one by one;
+// causal lengths (start + 1, start + 2, ...; the host keeps them inside the
+// cache) in closed form.
+__device__ __forceinline__ long long tiles_before(const Params& p, int b) {
+  if (!p.seq_lens) return causal_tile_sum(p, (long long)p.causal_base + b) -
+                          causal_tile_sum(p, p.causal_base);
+  long long t = 0;
+  for (int i = 0; i < b; ++i) t += req_tiles(p, i);
+  return t;
 }
 
 struct Segment {
@@ -170,8 +188,7 @@ struct Cursor {
 __device__ void seg_begin(const Params& p, int cl, Cursor& c) {
   c.idx = 0;
   if (p.mode == 0) {
-    long long T = 0;
-    for (int b = 0; b < p.B; ++b) T += req_tiles(p, b);
+    const long long T = tiles_before(p, p.B);
     // with fewer tiles than clusters only the first T clusters get work, so
     // that every cluster in a request's range has written its partial slot
     const long long P = min((long long)p.P, T);
@@ -183,6 +200,17 @@ __device__ void seg_begin(const Params& p, int cl, Cursor& c) {
     }
     c.b = 0;
     c.pre = 0;
+    if (!p.seq_lens && c.cur > 0) {
+      // causal lengths: the last request starting at or before tile c.cur,
+      // by bisection instead of a walk over all earlier requests
+      int lo = 0, hi = p.B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (tiles_before(p, mid) <= c.cur) lo = mid; else hi = mid - 1;
+      }
+      c.b = lo;
+      c.pre = tiles_before(p, lo);
+    }
   } else {
     c.b = cl / p.S;
     c.pre = c.cur = c.end = 0;
@@ -1416,7 +1444,10 @@ sm100_merge_kernel(const Params p) {
   const int h = blockIdx.y * kMergeHeads + warp;
   __shared__ long long red[2][kMergeHeads];
   long long pre = 0, tot = 0;
-  if (p.mode == 0) {  // tiles before request b and in total
+  if (p.mode == 0 && !p.seq_lens) {  // causal lengths: closed form
+    pre = tiles_before(p, b);
+    tot = tiles_before(p, p.B);
+  } else if (p.mode == 0) {  // tiles before request b and in total
     for (int bb = threadIdx.x; bb < p.B; bb += kMergeThreads) {
       const long long nt = req_tiles(p, bb);
       tot += nt;
@@ -1766,6 +1797,7 @@ cudaError_t launch_decode_sm100(const DecodeProblem& dp, int num_splits, void* w
 void fill_params(const DecodeProblem& dp, Params& p) {
   p = Params{};
   p.seq_lens = dp.seq_lens;
+  p.causal_base = dp.causal_base;
   p.page_table = dp.page_table;
   p.pt_sb = dp.pt_sb;
   p.num_blocks = (int)dp.num_blocks;

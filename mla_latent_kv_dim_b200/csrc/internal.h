@@ -22,7 +22,8 @@ struct DecodeProblem {
   int64_t c_s0, c_s1;      // paged: block, row strides; contiguous: batch, row
   int64_t num_blocks;      // paged only
   int64_t cache_rows;      // contiguous: Lmax;  paged: max_pages * 64
-  const int* seq_lens;     // [B]
+  const int* seq_lens;     // [B], or nullptr: request b holds causal_base + b + 1 tokens
+  int causal_base;
   const int* page_table;   // [B, max_pages] or nullptr (contiguous)
   int64_t pt_sb;
   int max_pages;
@@ -94,8 +95,9 @@ cudaError_t launch_rotate(void* x, int64_t B, int64_t H, int64_t sb, int64_t sh,
                           float* scratch, int64_t chunk_b, cudaStream_t stream);
 
 // ---------------------------------------------------------------- cache append
+// positions == nullptr: row b goes to position pos0 + b.
 cudaError_t launch_cache_append(const void* kv_new, int in_bf16, int64_t n_sb, const int* positions,
-                                const int* page_table, int64_t pt_sb, int max_pages,
+                                int pos0, const int* page_table, int64_t pt_sb, int max_pages,
                                 int64_t num_blocks, int64_t cap_rows, void* cache, int64_t c_s0,
                                 int64_t c_s1, int B, int groups, int hadamard, float eps,
                                 cudaStream_t stream);

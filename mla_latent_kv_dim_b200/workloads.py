@@ -14,6 +14,12 @@ Recipe (fixed order, one NumPy PCG64 stream per workload seed):
    of request b is physical block ``perm[first_page[b] + p]``;
 5. ``W_uv`` [H, 512, 128] ~ N(0, 0.02) when requested.
 
+Prefill inputs (``make_prefill_inputs``), one request: ``q`` [T, H, 576]
+~ N(0, 1); the prompt's new rows ``kv_new`` [T, 576] drawn like cache rows
+(float32, not rounded); a paged cache whose rows (the ``start`` tokens cached
+before the prompt, and unused rows) are drawn like cache rows; the request's
+page row is the first pages of ``rng.permutation(num_blocks)``.
+
 Values are drawn in float32 and rounded to bf16 (round-to-nearest-even).
 The named workloads are DeepSeek-V2-Lite, DeepSeek-V3 and Kimi-K2-shaped
 stand-ins (no checkpoints or datasets are used).
@@ -139,6 +145,33 @@ def make_inputs(B: int, H: int, lens, *, paged: bool = True, decay: bool = False
                     seq_lens=torch.from_numpy(seq.astype(np.int32)),
                     q=q, cache=cache, page_table=page_table, W_uv=W,
                     meta=dict(seed=seed, decay=decay, paged=paged))
+
+
+@dataclass
+class PrefillInputs:
+    start: int
+    q: torch.Tensor         # [T, H, 576] bf16
+    kv_new: torch.Tensor    # [T, 576] f32
+    cache: torch.Tensor     # [num_blocks, 64, 576] bf16
+    page_row: torch.Tensor  # [pages] int32
+    scale: float = SOFTMAX_SCALE
+
+
+def make_prefill_inputs(T: int, H: int, start: int = 0, *, seed: int = 0,
+                        spare_blocks: int = 1, decay: bool = True) -> PrefillInputs:
+    """One request's prompt of T tokens after ``start`` cached tokens."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    q = _to_bf16(rng.standard_normal((T, H, WIDTH), dtype=np.float32))
+    new = rng.standard_normal((T, WIDTH), dtype=np.float32)
+    if decay:
+        new[:, :LATENT] *= np.exp(-np.arange(LATENT, dtype=np.float64) / 128.0).astype(np.float32)
+    pages = max(1, (start + T + BLOCK - 1) // BLOCK)
+    nblk = pages + spare_blocks
+    cache = torch.empty((nblk, BLOCK, WIDTH), dtype=torch.bfloat16)
+    _draw_rows(rng, nblk * BLOCK, decay, cache)
+    row = rng.permutation(nblk)[:pages].astype(np.int32)
+    return PrefillInputs(start=start, q=q, kv_new=torch.from_numpy(new), cache=cache,
+                         page_row=torch.from_numpy(row))
 
 
 def make_workload(name: str, pin: bool = False, batch: int | None = None) -> Workload:

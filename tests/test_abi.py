@@ -309,3 +309,35 @@ def test_cache_append_validates_without_launch():
     assert call(eps=-1.0) == -1 and call(eps=float("nan")) == -1
     assert call(t=None) == -1                                     # contiguous: [B, Lmax, 576]
     assert tp.launch_count() == before
+
+
+def test_prefill_validates_without_launch():
+    L = tp.lib()
+    before = tp.launch_count()
+    B = ctypes.byref
+    q = _fake((5, 16, 576), torch.bfloat16)
+    new = _fake((5, 576), torch.bfloat16)
+    row = _fake((2,), torch.int32)
+    cache = _fake((10, 64, 576), torch.bfloat16)
+    out = _fake((5, 16, 512), torch.float32)
+
+    def call(q=q, n=new, start=0, r=row, c=cache, groups=1, had=0, eps=1e-6, scale=0.1, o=out,
+             ws=None, ws_bytes=0):
+        return L.tpla_prefill(B(q), B(n), start, B(r) if r is not None else None, B(c), groups,
+                              had, ctypes.c_float(eps), ctypes.c_float(scale), B(o), None, ws,
+                              ws_bytes, None)
+
+    assert call(n=_fake((4, 576), torch.bfloat16)) == -1        # one row per prompt token
+    assert call(n=_fake((5, 512), torch.bfloat16)) == -1        # row width
+    assert call(start=-1) == -1
+    assert call(start=124) == -1                                # 124 + 5 > 2 pages
+    assert call(r=None) == -1 and call(r=_fake((2, 2), torch.int32)) == -1
+    assert call(c=_fake((10, 32, 576), torch.bfloat16)) == -2   # 64-token pages only
+    assert call(groups=3) == -1 and call(had=2) == -1 and call(eps=-1.0) == -1
+    assert call(scale=float("inf")) == -1
+    assert call(o=_fake((5, 16, 256), torch.float32)) == -1     # out is [T, H, 512]
+    assert call(q=_fake((5, 16, 576), torch.float32)) == -1     # bf16 queries
+    assert call(q=_fake((1 << 20 + 1, 1, 576), torch.bfloat16)) == -2
+    n = ctypes.c_size_t(7)
+    assert L.tpla_prefill_workspace_size(None, B(n)) == -1
+    assert tp.launch_count() == before

@@ -3,11 +3,14 @@ Hadamard-rotated, RMS-normalised per shard, stored in the paged or contiguous
 cache) against the float64 oracle, through the C ABI.
 
 The kernel computes in f32 and rounds once to bf16; the oracle's float64 row
-rounded to bf16 (round-to-nearest-even) is the reference.  The two can differ
-only where the f32 value lies within rounding distance of a bf16 midpoint, so
-a stored value may differ from the rounded oracle by at most one bf16 step
-(relative 2^-7 bounds it) and almost all are equal.  Rows not written must be
-bit-identical to the cache before the call."""
+rounded to bf16 (round-to-nearest-even) is the reference.  The two differ
+where the f32 value lies within rounding distance of a bf16 midpoint (one
+bf16 step: relative 2^-7 bounds it), and, for the rare entries that the
+Hadamard sums cancel to nearly zero, by the f32 rounding of those sums
+itself: about 1e-6 on rows of unit RMS (a float32 restatement of the
+transform shows 7e-7), which the absolute floor 2^-16 covers.  Almost all
+stored values are equal.  Rows not written must be bit-identical to the
+cache before the call."""
 
 import numpy as np
 import pytest
@@ -49,7 +52,7 @@ def _check_rows(got, before, want16, written):
     assert np.array_equal(g[untouched], b[untouched]), "rows outside the positions changed"
     gw, ww = g[written], w[written]
     err = np.abs(gw - ww)
-    assert np.all(err <= 2.0 ** -7 * np.abs(ww) + 1e-30), f"max err {err.max()}"
+    assert np.all(err <= 2.0 ** -7 * np.abs(ww) + 2.0 ** -16), f"max err {err.max()}"
     assert np.mean(gw == ww) >= 0.99
 
 
