@@ -995,7 +995,8 @@ constexpr int kMiscBytes = kNumBars * 8 + 16;
 constexpr int kSmemBytes = 232448;  // the per-block maximum; the ring takes what Q leaves
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 64, false, true);
+__constant__ uint32_t kIdescPVn[2] = {idesc_bf16_f32(128, 64, false, true),
+                                      idesc_bf16_f32(128, 128, false, true)};
 
 struct Bars {
   uint32_t base;
@@ -1204,10 +1205,15 @@ __device__ void pv_issuer(const Params& p, int range, uint32_t sbase, uint32_t t
   Segment s;
   uint32_t n = 0, U = 0;
   const int nq = p.dq + 1;
-  // MN-major V operand: rows = tokens (K), 64 latent columns per 128-byte row
+  // MN-major V operand: rows = tokens (K), 64 latent columns per 128-byte
+  // row; chunks in consecutive slots form one operand whose 64-column groups
+  // lie one stage apart (the leading-byte offset)
   const uint64_t dV = sw128_desc(sbase + L.ring, kStage / 2, 1024);
+  const uint64_t dV2 = sw128_desc(sbase + L.ring, kStage, 1024);
   const uint32_t v_lo = (uint32_t)dV, v_hi = (uint32_t)(dV >> 32);
+  const uint32_t v2_lo = (uint32_t)dV2, v2_hi = (uint32_t)(dV2 >> 32);
   constexpr uint32_t kStageDesc = kStage >> 4;
+  const uint32_t ring = (uint32_t)p.ring;
   while (seg_next(p, range, cur, s)) {
     const int ntiles = s.t_hi - s.t_lo;
     if (ntiles == 0) continue;
@@ -1215,14 +1221,22 @@ __device__ void pv_issuer(const Params& p, int range, uint32_t sbase, uint32_t t
       if (!wait_bar(bars.p_full(U & 1), (U >> 1) & 1, abort_flag)) return;
       tc_fence_after();
       const uint32_t pa = tmem + kColS + 128 * (U & 1);  // P: 64 columns of bf16 pairs
-      for (int c = 0; c < p.dq; ++c) {
-        const uint32_t slot = (n + 1 + c) % (uint32_t)p.ring;
-        const uint32_t b = v_lo + slot * kStageDesc;
+      for (int c = 0; c < p.dq;) {
+        // the tile's next latent chunks, two at a time where their slots are
+        // consecutive, are one operand of N = 64 x run.  (Runs of four, N =
+        // 256, measured slower at G = 2: the first slot of a run is released
+        // only when the whole run is done.)
+        const uint32_t slot = (n + 1 + c) % ring;
+        const int run = min(min(p.dq - c, (int)(ring - slot)), 2);
         const uint32_t dO = tmem + kColO + 64 * c;
+        const uint32_t idesc = kIdescPVn[run - 1];
+        const uint32_t b = (run > 1 ? v2_lo : v_lo) + slot * kStageDesc;
+        const uint32_t bh = run > 1 ? v2_hi : v_hi;
 #pragma unroll
         for (int k = 0; k < 8; ++k)  // 16 tokens per step: P +8 columns, V +2 KB
-          mma_ts(dO, pa + 8 * k, b + 128 * k, v_hi, kIdescPV, (j | k) != 0);
-        commit(bars.empty(slot));
+          mma_ts(dO, pa + 8 * k, b + 128 * k, bh, idesc, (j | k) != 0);
+        for (int r = 0; r < run; ++r) commit(bars.empty(slot + r));
+        c += run;
       }
       commit(bars.pv_done(U & 1));
       n += nq;
