@@ -136,6 +136,7 @@ struct Params {
   int W;
   int tile_tok;  // tokens per schedule tile: 256 (pair kernel) or 128 (shard kernel)
   int ring;      // shard kernel: ring slots
+  int nS;        // shard kernel: S / P buffers in TMEM (2 or 3: 128 nS + d <= 512)
   int mode;  // 0 = balanced persistent ranges, 1 = explicit equal splits
   int P;     // clusters
   int S;     // explicit splits
@@ -988,9 +989,9 @@ constexpr int kMaxRing = 12;
 constexpr int kWarpQK = 0, kWarpPV = 1, kWarpProd0 = 2, kWarpSm0 = 4;  // producers: warps 2, 3
 constexpr int kSoftmaxWarps = 4;
 constexpr int kThreads = 32 * (kWarpSm0 + kSoftmaxWarps);
-constexpr uint32_t kColS = 0;    // S / P buffers: [0, 128), [128, 256)
-constexpr uint32_t kColO = 256;  // O: d <= 256 columns
-constexpr int kNumBars = 2 * kMaxRing + 8;
+constexpr uint32_t kColS = 0;    // S / P buffers: 128 columns each, nS of them
+constexpr int kMaxS = 3;         // O (d columns) follows them: 128 nS + d <= 512
+constexpr int kNumBars = 2 * kMaxRing + 2 + 3 * kMaxS;
 constexpr int kMiscBytes = kNumBars * 8 + 16;
 constexpr int kSmemBytes = 232448;  // the per-block maximum; the ring takes what Q leaves
 
@@ -1005,8 +1006,10 @@ struct Bars {
   __device__ uint32_t q_full() const { return base + 8 * (2 * kMaxRing); }
   __device__ uint32_t q_empty() const { return base + 8 * (2 * kMaxRing + 1); }
   __device__ uint32_t s_full(int i) const { return base + 8 * (2 * kMaxRing + 2 + i); }
-  __device__ uint32_t p_full(int i) const { return base + 8 * (2 * kMaxRing + 4 + i); }
-  __device__ uint32_t pv_done(int i) const { return base + 8 * (2 * kMaxRing + 6 + i); }
+  __device__ uint32_t p_full(int i) const { return base + 8 * (2 * kMaxRing + 2 + kMaxS + i); }
+  __device__ uint32_t pv_done(int i) const {
+    return base + 8 * (2 * kMaxRing + 2 + 2 * kMaxS + i);
+  }
 };
 
 struct Layout {  // shared-memory offsets (bytes from the 1 KB aligned base)
@@ -1151,6 +1154,7 @@ __device__ void qk_issuer(const Params& p, int range, int g, uint32_t sbase, uin
   seg_begin(p, range, cur);
   Segment s;
   uint32_t n = 0, qloads = 0, U = 0, parity = 0;
+  uint32_t si = 0, sph = 0;  // S buffer of tile U, parity of its use count
   const int nq = p.dq + 1;
   int rk0, rk1;
   rope_steps(p, g, rk0, rk1);
@@ -1166,10 +1170,10 @@ __device__ void qk_issuer(const Params& p, int range, int g, uint32_t sbase, uin
     ++qloads;
     tc_fence_after();
     for (int j = 0; j < ntiles; ++j, ++U) {
-      // S[U & 1] (with the P over it) is free once P.V of tile U - 2 completed
-      if (U >= 2 && !wait_bar(bars.pv_done(U & 1), ((U - 2) >> 1) & 1, abort_flag)) return;
+      // S buffer si (with the P over it) is free once P.V of tile U - nS completed
+      if (U >= (uint32_t)p.nS && !wait_bar(bars.pv_done(si), sph ^ 1u, abort_flag)) return;
       tc_fence_after();
-      const uint32_t dS = tmem + kColS + 128 * (U & 1);
+      const uint32_t dS = tmem + kColS + 128 * si;
       uint32_t acc = 0;
       for (int st = 0; st < nq; ++st) {
         const uint32_t slot = (n + st) % (uint32_t)p.ring;
@@ -1191,8 +1195,12 @@ __device__ void qk_issuer(const Params& p, int range, int g, uint32_t sbase, uin
           commit(bars.empty(slot));  // the rope chunk is needed by QK^T only
         }
       }
-      commit(bars.s_full(U & 1));
+      commit(bars.s_full(si));
       n += nq;
+      if (++si == (uint32_t)p.nS) {
+        si = 0;
+        sph ^= 1u;
+      }
     }
     commit(bars.q_empty());
   }
@@ -1204,6 +1212,8 @@ __device__ void pv_issuer(const Params& p, int range, uint32_t sbase, uint32_t t
   seg_begin(p, range, cur);
   Segment s;
   uint32_t n = 0, U = 0;
+  uint32_t si = 0, sph = 0;  // S / P buffer of tile U, parity of its use count
+  const uint32_t colO = kColS + 128 * (uint32_t)p.nS;
   const int nq = p.dq + 1;
   // MN-major V operand: rows = tokens (K), 64 latent columns per 128-byte
   // row; chunks in consecutive slots form one operand whose 64-column groups
@@ -1218,9 +1228,9 @@ __device__ void pv_issuer(const Params& p, int range, uint32_t sbase, uint32_t t
     const int ntiles = s.t_hi - s.t_lo;
     if (ntiles == 0) continue;
     for (int j = 0; j < ntiles; ++j, ++U) {
-      if (!wait_bar(bars.p_full(U & 1), (U >> 1) & 1, abort_flag)) return;
+      if (!wait_bar(bars.p_full(si), sph, abort_flag)) return;
       tc_fence_after();
-      const uint32_t pa = tmem + kColS + 128 * (U & 1);  // P: 64 columns of bf16 pairs
+      const uint32_t pa = tmem + kColS + 128 * si;  // P: 64 columns of bf16 pairs
       for (int c = 0; c < p.dq;) {
         // the tile's next latent chunks, two at a time where their slots are
         // consecutive, are one operand of N = 64 x run.  (Runs of four, N =
@@ -1228,7 +1238,7 @@ __device__ void pv_issuer(const Params& p, int range, uint32_t sbase, uint32_t t
         // only when the whole run is done.)
         const uint32_t slot = (n + 1 + c) % ring;
         const int run = min(min(p.dq - c, (int)(ring - slot)), 2);
-        const uint32_t dO = tmem + kColO + 64 * c;
+        const uint32_t dO = tmem + colO + 64 * c;
         const uint32_t idesc = kIdescPVn[run - 1];
         const uint32_t b = (run > 1 ? v2_lo : v_lo) + slot * kStageDesc;
         const uint32_t bh = run > 1 ? v2_hi : v_hi;
@@ -1238,8 +1248,12 @@ __device__ void pv_issuer(const Params& p, int range, uint32_t sbase, uint32_t t
         for (int r = 0; r < run; ++r) commit(bars.empty(slot + r));
         c += run;
       }
-      commit(bars.pv_done(U & 1));
+      commit(bars.pv_done(si));
       n += nq;
+      if (++si == (uint32_t)p.nS) {
+        si = 0;
+        sph ^= 1u;
+      }
     }
   }
 }
@@ -1250,10 +1264,15 @@ __device__ void softmax(const Params& p, int range, int i_sh, int g, uint32_t tm
   const int head = 32 * (w & 3) + (int)(threadIdx.x & 31);  // = this thread's TMEM lane
   const uint32_t lane_base = (uint32_t)(32 * (w & 3)) << 16;
   const int col_base = p.shard < 0 ? g * p.d : 0;
+  const uint32_t colO = kColS + 128 * (uint32_t)p.nS;
   Cursor cur;
   seg_begin(p, range, cur);
   Segment s;
   uint32_t U = 0;
+  uint32_t si = 0, sph = 0;  // S buffer of tile U, parity of its use count
+  // buffer and parity of tile U - 1 (the previous P.V)
+  auto prev_buf = [&]() { return si == 0 ? (uint32_t)p.nS - 1 : si - 1; };
+  auto prev_ph = [&]() { return si == 0 ? sph ^ 1u : sph; };
   while (seg_next(p, range, cur, s)) {
     const int ntiles = s.t_hi - s.t_lo;
     if (ntiles == 0) {  // empty chunk: out 0, lse -inf
@@ -1267,9 +1286,9 @@ __device__ void softmax(const Params& p, int range, int i_sh, int g, uint32_t tm
     float m = -INFINITY, l = 0.f;
     for (int j = 0; j < ntiles; ++j, ++U) {
       const int t = s.t_lo + j;
-      if (!wait_bar(bars.s_full(U & 1), (U >> 1) & 1, abort_flag)) return;
+      if (!wait_bar(bars.s_full(si), sph, abort_flag)) return;
       tc_fence_after();
-      const uint32_t sb = tmem + lane_base + kColS + 128 * (U & 1);
+      const uint32_t sb = tmem + lane_base + kColS + 128 * si;
       float x[128];
       {
         uint32_t r[4][32];
@@ -1309,10 +1328,10 @@ __device__ void softmax(const Params& p, int range, int i_sh, int g, uint32_t tm
       l *= factor;
       if (__any_sync(0xffffffffu, resc)) {
         // O was last written by P.V of tile U - 1 (not the first of the segment)
-        if (!wait_bar(bars.pv_done((U - 1) & 1), ((U - 1) >> 1) & 1, abort_flag)) return;
+        if (!wait_bar(bars.pv_done(prev_buf()), prev_ph(), abort_flag)) return;
         tc_fence_after();
         for (int c0 = 0; c0 < p.d; c0 += 32) {
-          const uint32_t ta = tmem + lane_base + kColO + c0;
+          const uint32_t ta = tmem + lane_base + colO + c0;
           uint32_t o[32];
           tmem_ld32(ta, o);
           tmem_wait_ld();
@@ -1345,16 +1364,20 @@ __device__ void softmax(const Params& p, int range, int i_sh, int g, uint32_t tm
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if ((threadIdx.x & 31) == 0) arrive(bars.p_full(U & 1));
+      if ((threadIdx.x & 31) == 0) arrive(bars.p_full(si));
+      if (++si == (uint32_t)p.nS) {
+        si = 0;
+        sph ^= 1u;
+      }
     }
     // epilogue: the segment's last P.V done
-    if (!wait_bar(bars.pv_done((U - 1) & 1), ((U - 1) >> 1) & 1, abort_flag)) return;
+    if (!wait_bar(bars.pv_done(prev_buf()), prev_ph(), abort_flag)) return;
     tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
     const float lse = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
     for (int c0 = 0; c0 < p.d; c0 += 32) {
       uint32_t o[32];
-      tmem_ld32(tmem + lane_base + kColO + c0, o);
+      tmem_ld32(tmem + lane_base + colO + c0, o);
       tmem_wait_ld();
       write_out_row(p, s, head, col_base + c0, reinterpret_cast<const float*>(o), inv);
     }
@@ -1384,7 +1407,7 @@ tpla_decode_shard_kernel(const __grid_constant__ CUtensorMap qmap,
     }
     mbar_init(bars.q_full(), 1);
     mbar_init(bars.q_empty(), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMaxS; ++i) {
       mbar_init(bars.s_full(i), 1);
       mbar_init(bars.p_full(i), kSoftmaxWarps);
       mbar_init(bars.pv_done(i), 1);
@@ -1933,6 +1956,9 @@ cudaError_t launch_decode_shard_group(const DecodeProblem& dp, int num_splits, v
   int ring = (shd::kSmemBytes - 1024 - q_bytes - shd::kMiscBytes) / shd::kStage;
   p.ring = ring > shd::kMaxRing ? shd::kMaxRing : ring;
   if (p.ring < 2) return cudaErrorNotSupported;
+  // TMEM holds nS S buffers of 128 columns and O (d columns): a third
+  // buffer fits for d <= 128 (G >= 4) and lets a third tile into flight
+  p.nS = (512 - p.d) / 128 < shd::kMaxS ? (512 - p.d) / 128 : shd::kMaxS;
   if (!set_schedule(dp, num_splits, num_ranges(dp, d), ws, ws_bytes, p))
     return cudaErrorInvalidValue;
   const int ctas = p.P * p.nsh;
