@@ -135,6 +135,7 @@ struct Params {
   float* part_l;  // [slots, H, nsh]
   int W;
   int tile_tok;  // tokens per schedule tile: 256 (pair kernel) or 128 (shard kernel)
+  int seg_cost;  // schedule cost of a segment's fixed work, in tiles
   int ring;      // shard kernel: ring slots
   int nS;        // shard kernel: S / P buffers in TMEM (2 or 3: 128 nS + d <= 512)
   int mode;  // 0 = balanced persistent ranges, 1 = explicit equal splits
@@ -163,14 +164,23 @@ __device__ __forceinline__ long long causal_tile_sum(const Params& p, long long 
   return tt * q * (q + 1) / 2 + r * (q + 1);
 }
 
-// Tiles of requests [0, b).  Lengths from seq_lens are summed one by one;
-// causal lengths (start + 1, start + 2, ...; the host keeps them inside the
-// cache) in closed form.
-__device__ __forceinline__ long long tiles_before(const Params& p, int b) {
-  if (!p.seq_lens) return causal_tile_sum(p, (long long)p.causal_base + b) -
-                          causal_tile_sum(p, p.causal_base);
+// Schedule cost of a request: its tiles plus seg_cost for the fixed work of
+// a segment (loading q, the epilogue), so that a range of many short
+// requests is not overloaded.  An empty request costs nothing.
+__device__ __forceinline__ long long req_cost(const Params& p, int b) {
+  const int nt = req_tiles(p, b);
+  return nt > 0 ? (long long)nt + p.seg_cost : 0;
+}
+
+// Cost of requests [0, b).  Lengths from seq_lens are summed one by one;
+// causal lengths (start + 1, start + 2, ...; never empty; the host keeps them
+// inside the cache) in closed form.
+__device__ __forceinline__ long long cost_before(const Params& p, int b) {
+  if (!p.seq_lens)
+    return causal_tile_sum(p, (long long)p.causal_base + b) - causal_tile_sum(p, p.causal_base) +
+           (long long)p.seg_cost * b;
   long long t = 0;
-  for (int i = 0; i < b; ++i) t += req_tiles(p, i);
+  for (int i = 0; i < b; ++i) t += req_cost(p, i);
   return t;
 }
 
@@ -189,9 +199,9 @@ struct Cursor {
 __device__ void seg_begin(const Params& p, int cl, Cursor& c) {
   c.idx = 0;
   if (p.mode == 0) {
-    const long long T = tiles_before(p, p.B);
-    // with fewer tiles than clusters only the first T clusters get work, so
-    // that every cluster in a request's range has written its partial slot
+    // range cl covers the cost positions [cl C / P, (cl + 1) C / P); with a
+    // smaller total cost than clusters only the first C clusters get work
+    const long long T = cost_before(p, p.B);
     const long long P = min((long long)p.P, T);
     if (cl >= P) {
       c.cur = c.end = 0;
@@ -202,15 +212,15 @@ __device__ void seg_begin(const Params& p, int cl, Cursor& c) {
     c.b = 0;
     c.pre = 0;
     if (!p.seq_lens && c.cur > 0) {
-      // causal lengths: the last request starting at or before tile c.cur,
-      // by bisection instead of a walk over all earlier requests
+      // causal lengths: the last request starting at or before position
+      // c.cur, by bisection instead of a walk over all earlier requests
       int lo = 0, hi = p.B - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) / 2;
-        if (tiles_before(p, mid) <= c.cur) lo = mid; else hi = mid - 1;
+        if (cost_before(p, mid) <= c.cur) lo = mid; else hi = mid - 1;
       }
       c.b = lo;
-      c.pre = tiles_before(p, lo);
+      c.pre = cost_before(p, lo);
     }
   } else {
     c.b = cl / p.S;
@@ -221,19 +231,28 @@ __device__ void seg_begin(const Params& p, int cl, Cursor& c) {
 __device__ bool seg_next(const Params& p, int cl, Cursor& c, Segment& s) {
   if (p.mode == 0) {
     if (c.cur >= c.end) return false;
-    while (c.b < p.B && c.pre + req_tiles(p, c.b) <= c.cur) {
-      c.pre += req_tiles(p, c.b);
+    while (c.b < p.B && c.pre + req_cost(p, c.b) <= c.cur) {
+      c.pre += req_cost(p, c.b);
       ++c.b;
     }
     if (c.b >= p.B) return false;
+    // request c.b: its fixed cost, then its tiles at positions t0, t0 + 1, ...
     const int nt = req_tiles(p, c.b);
+    const long long t0 = c.pre + p.seg_cost;
+    const long long lo = max(c.cur, t0), hi = min(c.end, t0 + nt);
+    if (lo >= hi) {  // the range ends inside the request's fixed cost
+      c.cur = c.end;
+      return false;
+    }
     s.b = c.b;
     s.L = req_len(p, c.b);
-    s.t_lo = (int)(c.cur - c.pre);
-    s.t_hi = (int)min((long long)nt, c.end - c.pre);
+    s.t_lo = (int)(lo - t0);
+    s.t_hi = (int)(hi - t0);
     s.complete = (s.t_lo == 0 && s.t_hi == nt);
+    // a range's first segment writes partials to slot 2 cl, the others
+    // (only its last can be partial) to 2 cl + 1
     s.slot = 2 * cl + (c.idx == 0 ? 0 : 1);
-    c.cur = c.pre + s.t_hi;
+    c.cur = hi;
     ++c.idx;
     return true;
   }
@@ -1482,13 +1501,13 @@ sm100_merge_kernel(const Params p) {
   __shared__ long long red[2][kMergeHeads];
   long long pre = 0, tot = 0;
   if (p.mode == 0 && !p.seq_lens) {  // causal lengths: closed form
-    pre = tiles_before(p, b);
-    tot = tiles_before(p, p.B);
-  } else if (p.mode == 0) {  // tiles before request b and in total
+    pre = cost_before(p, b);
+    tot = cost_before(p, p.B);
+  } else if (p.mode == 0) {  // schedule cost before request b and in total
     for (int bb = threadIdx.x; bb < p.B; bb += kMergeThreads) {
-      const long long nt = req_tiles(p, bb);
-      tot += nt;
-      if (bb < b) pre += nt;
+      const long long nc = req_cost(p, bb);
+      tot += nc;
+      if (bb < b) pre += nc;
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
@@ -1511,9 +1530,10 @@ sm100_merge_kernel(const Params p) {
   int s_lo = 0, s_hi = 0;  // cluster range of request b
   const long long P = min((long long)p.P, T);  // clusters that received work
   if (nt > 0) {
-    if (p.mode == 0) {
-      s_lo = (int)(((pre + 1) * P + T - 1) / T - 1);
-      s_hi = (int)(((pre + nt) * P + T - 1) / T - 1);
+    if (p.mode == 0) {  // the ranges holding the request's first and last tile
+      const long long x0 = pre + p.seg_cost;
+      s_lo = (int)(((x0 + 1) * P + T - 1) / T - 1);
+      s_hi = (int)(((x0 + nt) * P + T - 1) / T - 1);
       if (s_lo == s_hi) return;  // one cluster wrote the final result
     } else {
       if (p.S == 1) return;
@@ -1546,8 +1566,8 @@ sm100_merge_kernel(const Params p) {
     return;
   }
   // Slot of range c's partial of this request: 2c, except the first range,
-  // which used its second slot when the request started inside it (the one
-  // 64-bit division is done once here).
+  // which used its second slot when it began before the request (an earlier
+  // request's tiles came first; the one 64-bit division is done once here).
   const int first_slot = (p.mode == 0 && (long long)s_lo * T / P < pre) ? 2 * s_lo + 1 : 2 * s_lo;
   auto slot_of = [&](int c) -> int { return c == s_lo ? first_slot : 2 * c; };
   // Column groups of this lane: 16-byte groups 4 * lane + 128 * i of each
@@ -1924,6 +1944,7 @@ cudaError_t launch_decode_sm100_group(const DecodeProblem& dp, int num_splits, v
   p.qk_slots = dp.G == 2 ? 4 : 3;
   p.pv_slots = kRingSlots - p.qk_slots;
   p.tile_tok = kTileTok;
+  p.seg_cost = 1;  // q load and epilogue: about one 256-token tile
   if (!set_schedule(dp, num_splits, d.max_clusters, ws, ws_bytes, p)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
@@ -1951,6 +1972,7 @@ cudaError_t launch_decode_shard_group(const DecodeProblem& dp, int num_splits, v
   Params p;
   fill_params(dp, p);
   p.tile_tok = shd::kTile;
+  p.seg_cost = 2;  // q load and epilogue: about two 128-token tiles
   // the ring takes the shared memory the shard's q leaves
   const int q_bytes = (p.dq + 1) * shd::kQChunkBytes;
   int ring = (shd::kSmemBytes - 1024 - q_bytes - shd::kMiscBytes) / shd::kStage;
