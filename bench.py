@@ -63,6 +63,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--batch", type=int, default=None,
                     help="fewer requests of the same shape (profiling captures)")
+    ap.add_argument("--prefill", type=int, default=0,
+                    help="with --profile: time tpla_prefill of one prompt of this many "
+                         "tokens (H = 128) instead of the decode")
     ap.add_argument("--profile", action="store_true",
                     help="decode launches only: warmup + steps, one short JSON line")
     return ap.parse_args()
@@ -760,9 +763,37 @@ def _sm100_used(tp, q, cache, seq, pt, G, rope, out, args):
 
 
 def run_profile(args):
-    """Decode launches only (for ncu captures): W warm-up + K timed launches."""
+    """Decode launches only (for ncu captures): W warm-up + K timed launches.
+    With --prefill T: prefill calls of one T-token prompt instead."""
     import mla_latent_kv_dim_b200 as tp
     dev = torch.device("cuda", 0)
+    if args.prefill > 0:
+        from mla_latent_kv_dim_b200.workloads import make_prefill_inputs
+        T = args.prefill
+        pw = make_prefill_inputs(T, 128, 0, seed=31)
+        q, new, row, cache = pw.q.to(dev), pw.kv_new.to(dev), pw.page_row.to(dev), pw.cache.to(dev)
+        out = torch.empty((T, 128, LATENT), dtype=torch.float32, device=dev)
+        lse = torch.empty((T, 128, 1), dtype=torch.float32, device=dev)
+        ws = torch.empty(1 << 24, dtype=torch.uint8, device=dev)
+
+        def call():
+            tp.prefill(q, new, 0, row, cache, scale=pw.scale, out=out, lse=lse, workspace=ws)
+
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            call()
+        b.record()
+        torch.cuda.synchronize()
+        t = a.elapsed_time(b) / 1e3 / args.steps
+        fl = T * (T + 1) // 2 * 128 * flops_per_token_head(1)
+        print(json.dumps({"profile": "prefill", "T": T, "prefill_us": round(t * 1e6, 1),
+                          "tensor_tflops": round(fl / t / 1e12, 1),
+                          "status": tp.device_status()}), flush=True)
+        return 0
     w = make_workload(args.config, batch=args.batch)
     q, cache, seq = w.q.to(dev), w.cache.to(dev), w.seq_lens.to(dev)
     pt = None if w.page_table is None else w.page_table.to(dev)

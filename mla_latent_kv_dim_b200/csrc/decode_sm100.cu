@@ -1944,7 +1944,7 @@ cudaError_t launch_decode_sm100_group(const DecodeProblem& dp, int num_splits, v
   p.qk_slots = dp.G == 2 ? 4 : 3;
   p.pv_slots = kRingSlots - p.qk_slots;
   p.tile_tok = kTileTok;
-  p.seg_cost = 1;  // q load and epilogue: about one 256-token tile
+  p.seg_cost = 2;  // q load and epilogue (measured best of 1-3 on prompt prefill)
   if (!set_schedule(dp, num_splits, d.max_clusters, ws, ws_bytes, p)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
@@ -1972,7 +1972,7 @@ cudaError_t launch_decode_shard_group(const DecodeProblem& dp, int num_splits, v
   Params p;
   fill_params(dp, p);
   p.tile_tok = shd::kTile;
-  p.seg_cost = 2;  // q load and epilogue: about two 128-token tiles
+  p.seg_cost = 2;  // q load and epilogue (measured best of 2-6 on mixed lengths)
   // the ring takes the shared memory the shard's q leaves
   const int q_bytes = (p.dq + 1) * shd::kQChunkBytes;
   int ring = (shd::kSmemBytes - 1024 - q_bytes - shd::kMiscBytes) / shd::kStage;
