@@ -532,6 +532,7 @@ def run_ours(args):
 
     # ---- per-G decode-only sweep (vs G), full and one-shard
     vs_G = []
+    tp_rank = None
     clk_extras = None
     if not args.no_extras:
         cs = ClockSampler(local)
@@ -559,6 +560,25 @@ def run_ours(args):
                          "hbm_frac": round(nb / t / 1e9 / hbm_peak, 4),
                          "tok_s_layer": round(B / t, 1)})
             del o2, l2
+        # one tensor-parallel rank's step (its one-shard decode + its partial V
+        # up-projection, K = 512/G), against the exact-MLA step on one GPU
+        # (G = 1 decode + V-up); the all-reduce of y between ranks is not timed
+        from mla_latent_kv_dim_b200 import tensor_parallel as TPar
+        tp_rank = []
+        for GG in (1, 2, 4):
+            def rank_step():
+                TPar.rank_partial(q, cache, seq, pt, GG, 0, W, w.scale, rope, workspace=ws)
+            for _ in range(3):
+                rank_step()
+            a = torch.cuda.Event(enable_timing=True)
+            bb = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(50):
+                rank_step()
+            bb.record(stream)
+            torch.cuda.synchronize()
+            tp_rank.append({"G": GG, "rank_step_us": round(a.elapsed_time(bb) / 50 * 1e3, 1),
+                            "bytes": w.latent_kv_bytes(GG, 0 if GG > 1 else None, rope)})
         clk_extras = cs.stop()
 
     configs = None
@@ -592,6 +612,7 @@ def run_ours(args):
         "hbm_frac_step": round(value / world / hbm_peak, 4),
         "roofline": roof, "vs_G": vs_G, "vs_G_clocks": clk_extras,
         "one_shard_speedup_vs_mla": one_shard_speedups(vs_G),
+        "tp_rank_step": tp_rank,
         "configs": configs,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,

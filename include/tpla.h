@@ -242,8 +242,11 @@ TPLA_API int tpla_hadamard_apply(tpla_tensor* buf, int dim, tpla_stream_t stream
  * The V up-projection; with shard outputs laid side by side in latent space,
  * the contraction over j is the sum over shards that the tensor-parallel
  * all-reduce performs (feature request, "Directions under investigation").
- *   out_latent [B, H, 512] f32 or bf16;  W_uv [H, 512, Dv] bf16, Dv a
- *   multiple of 16 and <= 256;  y [B, H, Dv] f32.
+ *   out_latent [B, H, K] f32 or bf16;  W_uv [H, K, Dv] bf16, Dv a multiple
+ *   of 16 and <= 256;  y [B, H, Dv] f32.  K = 512 (the whole latent) or any
+ *   multiple of 64 up to 512: with K = 512 / G, the one-shard output of
+ *   rank g (tpla_decode_ex with opts->shard = g) and the rows I_g of W_uv
+ *   give that rank's partial product, which the all-reduce sums.
  * Accumulation is f32 on tensor cores; an f32 out_latent is split into two
  * bf16 terms (hi + lo) so that its rounding does not limit accuracy.
  */

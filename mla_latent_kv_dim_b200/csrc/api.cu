@@ -383,10 +383,11 @@ int tpla_vup_combine(const tpla_tensor* out_latent, const tpla_tensor* W_uv, tpl
                      tpla_stream_t stream) {
   if (!out_latent || (out_latent->dtype != TPLA_F32 && out_latent->dtype != TPLA_BF16))
     return TPLA_ERR_INVALID_ARG;
-  if (!check_tensor(out_latent, out_latent->dtype, 3) || out_latent->shape[2] != kLatent)
-    return TPLA_ERR_INVALID_ARG;
-  const int64_t B = out_latent->shape[0], H = out_latent->shape[1];
-  if (!check_tensor(W_uv, TPLA_BF16, 3) || W_uv->shape[0] != H || W_uv->shape[1] != kLatent)
+  if (!check_tensor(out_latent, out_latent->dtype, 3)) return TPLA_ERR_INVALID_ARG;
+  // K latent columns: 512, or one shard's 512 / G (a rank's partial product)
+  const int64_t B = out_latent->shape[0], H = out_latent->shape[1], K = out_latent->shape[2];
+  if (K < 64 || K > kLatent || K % 64) return TPLA_ERR_INVALID_ARG;
+  if (!check_tensor(W_uv, TPLA_BF16, 3) || W_uv->shape[0] != H || W_uv->shape[1] != K)
     return TPLA_ERR_INVALID_ARG;
   const int64_t Dv = W_uv->shape[2];
   if (Dv % 16 != 0 || Dv < 16 || Dv > 256) return TPLA_ERR_UNSUPPORTED;
@@ -400,7 +401,7 @@ int tpla_vup_combine(const tpla_tensor* out_latent, const tpla_tensor* W_uv, tpl
                              out_latent->stride[0], out_latent->stride[1], W_uv->data,
                              W_uv->stride[0], W_uv->stride[1],
                              reinterpret_cast<float*>(y->data), y->stride[0], y->stride[1],
-                             (int)B, (int)H, (int)Dv, reinterpret_cast<cudaStream_t>(stream));
+                             (int)B, (int)H, (int)Dv, (int)K, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? TPLA_OK : cuda_fail(e);
 }
 

@@ -80,7 +80,7 @@ bool vup_supported(const void* out_latent, int out_bf16, int64_t o_sb, int64_t o
                    const void* W, int64_t w_sh, int64_t w_sj);
 cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64_t o_sh,
                        const void* W, int64_t w_sh, int64_t w_sj, float* y,
-                       int64_t y_sb, int64_t y_sh, int B, int H, int Dv,
+                       int64_t y_sb, int64_t y_sh, int B, int H, int Dv, int K,
                        cudaStream_t stream);
 
 // ---------------------------------------------------------------- PCA reparameterisation

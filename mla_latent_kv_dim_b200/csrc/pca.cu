@@ -154,7 +154,7 @@ cudaError_t rotate_rows_f32(const __nv_bfloat16* x, int64_t rs, int64_t n, const
   for (int half = 0; half < 2; ++half) {
     cudaError_t e = launch_vup(x, 1, rs, rs, u + 256 * half, (int64_t)kLatent * kLatent,
                                kLatent, scratch + 256 * half, kLatent, kLatent, (int)n, 1, 256,
-                               stream);
+                               kLatent, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

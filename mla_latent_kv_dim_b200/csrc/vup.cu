@@ -1,4 +1,6 @@
-// V up-projection combine: y[b, h, :] = sum_j out[b, h, j] W_uv[h, j, :].
+// V up-projection combine: y[b, h, :] = sum_j out[b, h, j] W_uv[h, j, :],
+// over j < K (K = 512 for the whole latent; K = 512 / G for one rank's
+// shard, whose partial product the tensor-parallel all-reduce sums).
 //
 // In TPLA the shard outputs are combined by the existing o_proj all-reduce
 // (feature request "Bandwidth-optimal tensor-parallel sharding of MLA",
@@ -40,7 +42,7 @@ namespace {
 using namespace ptx;
 
 constexpr int kKC = 64;                   // latent columns per K chunk
-constexpr int kKChunks = kLatent / kKC;   // 8
+constexpr int kMaxKChunks = kLatent / kKC;  // 8
 constexpr int kMaxN = 64;                 // batch rows per CTA (MMA N)
 constexpr int kWBox = 8192;               // one [64 j][64 v] bf16 tile
 constexpr int kConvStages = 2;
@@ -55,6 +57,7 @@ struct VupParams {
   float* y;
   int64_t y_sb, y_sh;
   int B, H, Dv;
+  int kc;          // K chunks of 64 latent columns (K / 64, 1 .. 8)
   int mh;          // 128-row halves of Dv (1 or 2)
   int nt;          // batch rows per tile (MMA N), multiple of 16, <= 64
   int out_bf16;
@@ -175,7 +178,7 @@ vup_sm100_kernel(const __grid_constant__ CUtensorMap wmap,
       tma_prefetch(&omap);
     }
     int issued = 0;
-    for (int k = 0; k < kKChunks; ++k) {
+    for (int k = 0; k < p.kc; ++k) {
       const int s = k % R;
       int ok = 1;
       if (lane == 0) {
@@ -205,7 +208,7 @@ vup_sm100_kernel(const __grid_constant__ CUtensorMap wmap,
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, p.nt, true, false);
       bool ok = true;
-      for (int k = 0; k < kKChunks && ok; ++k) {
+      for (int k = 0; k < p.kc && ok; ++k) {
         const int s = k % R, c = k % kConvStages;
         ok = wait(raw_full(s), (k / R) & 1, abort_flag);
         if (ok && !p.out_bf16) ok = wait(conv_full(c), (k / kConvStages) & 1, abort_flag);
@@ -242,7 +245,7 @@ vup_sm100_kernel(const __grid_constant__ CUtensorMap wmap,
     bool ok = true;
     if (!p.out_bf16) {
       const int items = p.nt * 8;  // (row, 8-column group) per chunk
-      for (int k = 0; k < kKChunks && ok; ++k) {
+      for (int k = 0; k < p.kc && ok; ++k) {
         const int s = k % R, c = k % kConvStages;
         ok = wait(raw_full(s), (k / R) & 1, abort_flag);
         if (ok && k >= kConvStages) ok = wait(conv_empty(c), ((k / kConvStages) - 1) & 1, abort_flag);
@@ -320,9 +323,10 @@ bool vup_supported(const void* out_latent, int out_bf16, int64_t o_sb, int64_t o
 
 cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64_t o_sh,
                        const void* W, int64_t w_sh, int64_t w_sj, float* y, int64_t y_sb,
-                       int64_t y_sh, int B, int H, int Dv, cudaStream_t stream) {
+                       int64_t y_sh, int B, int H, int Dv, int K, cudaStream_t stream) {
   if (B == 0 || H == 0 || Dv == 0) return cudaSuccess;
-  if (!vup_supported(out_latent, out_bf16, o_sb, o_sh, W, w_sh, w_sj) || Dv > 256 || Dv % 16)
+  if (!vup_supported(out_latent, out_bf16, o_sb, o_sh, W, w_sh, w_sj) || Dv > 256 || Dv % 16 ||
+      K < kKC || K > kLatent || K % kKC)
     return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -337,6 +341,7 @@ cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64
   p.B = B;
   p.H = H;
   p.Dv = Dv;
+  p.kc = K / kKC;
   p.mh = Dv > 128 ? 2 : 1;
   p.nt = B >= kMaxN ? kMaxN : ((B + 15) / 16) * 16;
   p.out_bf16 = out_bf16;
@@ -353,10 +358,10 @@ cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64
   p.off_bar = p.off_conv + conv_bytes;
   const uint32_t smem = p.off_bar + 8 * (2 * kMaxRaw + 2 * kConvStages + 1) + 16 + 1024;
 
-  // W as [H][512][Dv] (v innermost): boxes of 64 v x 64 j, MN-major for the MMA
+  // W as [H][K][Dv] (v innermost): boxes of 64 v x 64 j, MN-major for the MMA
   CUtensorMap wmap, omap;
   {
-    cuuint64_t dims[3] = {(cuuint64_t)Dv, (cuuint64_t)kLatent, (cuuint64_t)H};
+    cuuint64_t dims[3] = {(cuuint64_t)Dv, (cuuint64_t)K, (cuuint64_t)H};
     cuuint64_t strides[2] = {(cuuint64_t)w_sj * 2, (cuuint64_t)w_sh * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)kKC, 1};
     cuuint32_t es[3] = {1, 1, 1};
@@ -366,10 +371,10 @@ cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  // out as [B][H][512] (j innermost): boxes of 64 j x 1 head x nt requests
+  // out as [B][H][K] (j innermost): boxes of 64 j x 1 head x nt requests
   {
     const uint64_t esz = out_bf16 ? 2 : 4;
-    cuuint64_t dims[3] = {(cuuint64_t)kLatent, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)H, (cuuint64_t)B};
     cuuint64_t strides[2] = {(cuuint64_t)o_sh * esz, (cuuint64_t)o_sb * esz};
     cuuint32_t box[3] = {(cuuint32_t)kKC, 1, (cuuint32_t)p.nt};
     cuuint32_t es[3] = {1, 1, 1};

@@ -209,6 +209,14 @@ def test_hadamard_and_vup_validation():
     W = _fake((3, 512, 128), torch.bfloat16)
     y = _fake((2, 4, 128), torch.float32)
     assert L.tpla_vup_combine(ctypes.byref(o), ctypes.byref(W), ctypes.byref(y), None) == -1
+    # K (the contracted latent columns): a multiple of 64 up to 512, shared by out and W
+    for K in (0, 32, 96, 576):
+        oK = _fake((2, 4, K), torch.float32)
+        WK = _fake((4, K, 128), torch.bfloat16)
+        assert L.tpla_vup_combine(ctypes.byref(oK), ctypes.byref(WK), ctypes.byref(y), None) == -1
+    o256 = _fake((2, 4, 256), torch.float32)
+    assert L.tpla_vup_combine(ctypes.byref(o256), ctypes.byref(_fake((4, 512, 128), torch.bfloat16)),
+                              ctypes.byref(y), None) == -1
     assert tp.launch_count() == 0
 
 
