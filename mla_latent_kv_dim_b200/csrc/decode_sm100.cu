@@ -1495,6 +1495,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __global__ void __launch_bounds__(kMergeThreads)
 sm100_merge_kernel(const Params p) {
+  // every block waits for the decode grid (launched as its programmatic
+  // dependent), so that this grid cannot finish before the decode has
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y * kMergeHeads + warp;
@@ -1910,12 +1913,23 @@ bool set_schedule(const DecodeProblem& dp, int num_splits, int ranges, void* ws,
   return true;
 }
 
+// The merge is launched as a programmatic dependent of the decode kernel:
+// its blocks are scheduled as the decode's CTAs retire and wait (griddepcontrol)
+// for the whole decode grid and its writes before reading anything.
 cudaError_t launch_merge(const DecodeProblem& dp, const Params& p, cudaStream_t stream) {
   if (p.mode == 1 && p.S == 1) return cudaSuccess;
-  sm100_merge_kernel<<<dim3(dp.B, (dp.H + kMergeHeads - 1) / kMergeHeads), kMergeThreads, 0,
-                       stream>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(dp.B, (dp.H + kMergeHeads - 1) / kMergeHeads);
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, sm100_merge_kernel, p);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_decode_sm100_group(const DecodeProblem& dp, int num_splits, void* ws,

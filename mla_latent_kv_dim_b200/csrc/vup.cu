@@ -165,6 +165,10 @@ vup_sm100_kernel(const __grid_constant__ CUtensorMap wmap,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  // launched as a programmatic dependent of the kernel before it (the merge
+  // or the decode that wrote `out`): the set-up above overlaps its end, and
+  // nothing is read before that grid and its writes are complete
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -397,10 +401,19 @@ cudaError_t launch_vup(const void* out_latent, int out_bf16, int64_t o_sb, int64
       g_vup_attr[dev & 63] = true;
     }
   }
-  dim3 grid(H, (B + p.nt - 1) / p.nt);
-  vup_sm100_kernel<<<grid, kThreads, smem, stream>>>(wmap, omap, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(H, (B + p.nt - 1) / p.nt);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, vup_sm100_kernel, wmap, omap, p);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t status_read_clear_vup(int* code) {
