@@ -1577,6 +1577,59 @@ sm100_merge_kernel(const Params p) {
   // shard (cw <= 512, so at most four).  Loads of two slots x all groups go
   // out together before the multiply-adds.
   const int ngrp = (cw + 127) / 128;
+  if (s_hi == s_lo + 1 && p.nsh * ngrp <= 4) {
+    // The usual case, a request cut once: two slots.  Every shard's lse and
+    // row groups of both slots are loaded before any is used, so the merge
+    // costs one round trip to memory instead of two per shard.
+    const int sa = first_slot, sb = 2 * s_hi;
+    const int nj = p.nsh * ngrp;
+    float4 oa[4], ob[4];
+    float la[4], lb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      oa[j] = ob[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      la[j] = lb[j] = -INFINITY;
+      if (j < nj) {
+        const int k = j / ngrp, i = j - k * ngrp;
+        if (4 * lane + 128 * i < cw) {
+          const int64_t col = (int64_t)h * p.W + k * cw + 4 * lane + 128 * i;
+          oa[j] = __ldcg(reinterpret_cast<const float4*>(p.part_o + (int64_t)sa * p.H * p.W + col));
+          ob[j] = __ldcg(reinterpret_cast<const float4*>(p.part_o + (int64_t)sb * p.H * p.W + col));
+        }
+      }
+      if (j < p.nsh) {
+        la[j] = __ldcg(p.part_l + ((int64_t)sa * p.H + h) * p.nsh + j);
+        lb[j] = __ldcg(p.part_l + ((int64_t)sb * p.H + h) * p.nsh + j);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (k >= p.nsh) break;
+      const float M = fmaxf(la[k], lb[k]);
+      float total = -INFINITY, wa = 0.f, wb = 0.f;
+      if (M != -INFINITY) {
+        total = M + logf(expf(la[k] - M) + expf(lb[k] - M));
+        wa = la[k] == -INFINITY ? 0.f : expf(la[k] - total);
+        wb = lb[k] == -INFINITY ? 0.f : expf(lb[k] - total);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (j < nj && j / ngrp == k) {
+          const int i = j - k * ngrp;
+          if (4 * lane + 128 * i < cw) {
+            // a slot of weight 0 contributes nothing, whatever its row holds
+            const float4 a = wa != 0.f ? oa[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 c = wb != 0.f ? ob[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+            write4(k * cw + 4 * lane + 128 * i,
+                   make_float4(fmaf(wb, c.x, wa * a.x), fmaf(wb, c.y, wa * a.y),
+                               fmaf(wb, c.z, wa * a.z), fmaf(wb, c.w, wa * a.w)));
+          }
+        }
+      }
+      write_lse(k, total);
+    }
+    return;
+  }
   for (int k = 0; k < p.nsh; ++k) {
     auto lse_of = [&](int c) { return __ldcg(p.part_l + ((int64_t)slot_of(c) * p.H + h) * p.nsh + k); };
     auto row_of = [&](int c) {
