@@ -29,7 +29,13 @@
  *     is owned by the caller.  The library never frees or retains pointers.
  *   - Every call is asynchronous on `stream` (NULL = legacy default stream)
  *     and performs no host synchronisation, except tpla_get_device_status.
- *   - Inputs are never modified, except the buffer of tpla_hadamard_apply.
+ *   - Inputs are never modified, except the buffer of tpla_hadamard_apply
+ *     and the cache of tpla_cache_append / tpla_prefill.
+ *   - Some kernels after the first of a call (the split-KV merge, the V
+ *     up-projection) are launched as programmatic dependents of the kernel
+ *     before them in the stream: they start their set-up early and read
+ *     nothing before that kernel has finished and its writes are visible.
+ *     Stream order, as the caller sees it, is unchanged.
  *   - Return value: TPLA_OK (0) or a negative tpla_status.  Arguments are
  *     validated before anything is launched; on an argument error nothing is
  *     launched and no memory is touched.  No C++ exception crosses the ABI.
