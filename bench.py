@@ -533,6 +533,7 @@ def run_ours(args):
     # ---- per-G decode-only sweep (vs G), full and one-shard
     vs_G = []
     tp_rank = None
+    setup = None
     clk_extras = None
     if not args.no_extras:
         cs = ClockSampler(local)
@@ -580,6 +581,7 @@ def run_ours(args):
             tp_rank.append({"G": GG, "rank_step_us": round(a.elapsed_time(bb) / 50 * 1e3, 1),
                             "bytes": w.latent_kv_bytes(GG, 0 if GG > 1 else None, rope)})
         clk_extras = cs.stop()
+        setup = setup_ops(tp, dev, cache, w.cache, hbm_peak)
 
     configs = None
     if not args.no_extras and not args.no_configs and world == 1:
@@ -613,6 +615,7 @@ def run_ours(args):
         "roofline": roof, "vs_G": vs_G, "vs_G_clocks": clk_extras,
         "one_shard_speedup_vs_mla": one_shard_speedups(vs_G),
         "tp_rank_step": tp_rank,
+        "setup_ops": setup,
         "configs": configs,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -724,6 +727,73 @@ def other_workloads(tp, dev, hbm_peak, tc_peak):
         del q, cache, seq, pt, W
         torch.cuda.empty_cache()
     del flush
+    return res
+
+
+def _median_us(fn, n, warm=2):
+    for _ in range(warm):
+        fn()
+    ts = []
+    for _ in range(n):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median([x.elapsed_time(z) for x, z in ts]) * 1e3
+
+
+def setup_ops(tp, dev, cache, host_cache, hbm_peak):
+    """The steps around the decode on the DeepSeek-V3 workload, each the
+    median of a few calls timed with CUDA events: the Hadamard rotation of
+    the whole stored cache (one-off; an even number of calls leaves it as it
+    was), the cache append of one decode step's 64 new rows and of a
+    65536-row batch (f32 rows in, Hadamard, two norm groups), and the PCA
+    calibration covariance over 262144 unrotated cache rows and the PCA
+    rotation of those rows, with the eigenvalue-sum shares of the G = 2 and
+    G = 4 shards (Eq. 25's alpha and beta) as information."""
+    res = {}
+    nb = cache.numel() // WIDTH * LATENT * 2  # the latent columns, read and written once
+    t = _median_us(lambda: tp.hadamard_apply(cache, LATENT), 4)
+    res["hadamard_cache"] = {"bytes": 2 * nb, "us": round(t, 1),
+                             "GB_s": round(2 * nb / t / 1e3, 1),
+                             "hbm_frac": round(2 * nb / t / 1e3 / hbm_peak, 4)}
+    g = torch.Generator().manual_seed(77)
+    for rows in (64, 65536):
+        blocks = (rows + 63) // 64
+        dst = torch.zeros((blocks, 64, WIDTH), dtype=torch.bfloat16, device=dev)
+        new = torch.randn((rows, WIDTH), generator=g).to(dev)
+        pt = torch.arange(blocks, dtype=torch.int32, device=dev).repeat_interleave(64)[:rows]
+        pt = pt.reshape(rows, 1).contiguous()
+        pos = (torch.arange(rows, dtype=torch.int32) % 64).to(dev)
+        t = _median_us(lambda: tp.cache_append(new, pos, pt, dst, norm_groups=2, hadamard=True), 20)
+        by = rows * WIDTH * (4 + 2)
+        res[f"append_{rows}"] = {"rows": rows, "bytes": by, "us": round(t, 2),
+                                 "GB_s": round(by / t / 1e3, 1),
+                                 "hbm_frac": round(by / t / 1e3 / hbm_peak, 4)}
+        del dst, new, pt, pos
+    n = 262144
+    rows = host_cache.view(-1, WIDTH)[:n].to(dev)
+    mean, cov = tp.latent_covariance(rows)
+    t = _median_us(lambda: tp.latent_covariance(rows), 5)
+    fl = 2.0 * n * LATENT * LATENT
+    res["pca_covariance"] = {"rows": n, "us": round(t, 1),
+                             "GB_s": round(rows.numel() * 2 / t / 1e3, 1),
+                             "fma_tflops": round(fl / t / 1e6, 2)}
+    lam, vec = torch.linalg.eigh(cov.double().cpu())
+    order = torch.argsort(lam, descending=True)
+    lam, vec = lam[order], vec[:, order]
+    U = vec.to(torch.bfloat16).contiguous().to(dev)
+    t = _median_us(lambda: tp.rotate_apply(rows, U), 5)
+    res["pca_rotate"] = {"rows": n, "us": round(t, 1),
+                         "GB_s": round(2 * rows.numel() * 2 / t / 1e3, 1)}
+    tot = float(lam.sum())
+    res["pca_shares"] = {f"G{G}": [round(float(lam[i * (LATENT // G):(i + 1) * (LATENT // G)].sum())
+                                         / tot, 4) for i in range(G)] for G in (2, 4)}
+    del rows, U
+    torch.cuda.empty_cache()
     return res
 
 
